@@ -1,0 +1,247 @@
+"""Seeded synthetic inputs for the exact-attention workloads.
+
+This module only draws random numbers and lays them out: sequence lengths,
+packed Q/K/V tensors, the page pool and its block table.  It holds none of
+the attention arithmetic, so the CUDA path and the CPU oracle can both be fed
+from it without sharing any of the method.
+
+Recipe (every workload): a ``torch.Generator`` on the CPU seeded with the
+workload's seed draws, in this order, (1) sequence/context lengths, (2) the
+page permutation (paged workloads), (3) q, (4) k, (5) v.  Values are fp32
+N(0, 1) rounded to bf16 (round-to-nearest-even); the fp32 originals are kept
+where a workload also needs them.  Large tensors are drawn in fixed-size
+chunks in a fixed order, so the bits depend only on the seed.
+
+Workload shapes follow the pages' cases: head_dim 128 at sequence length
+2048 (skill page appendix "performance reference"), 32 query heads over 8
+kv heads (skill page, GQA/MQA appendix), packed varlen batches described by
+cu_seqlens (skill page section 3.4), and paged KV caches addressed by a
+block table (skill page, PagedAttention appendix).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+_CHUNK = 1 << 24
+
+
+def randn_f32(shape, gen: torch.Generator) -> torch.Tensor:
+    """fp32 N(0,1) of ``shape``, drawn in fixed chunks so the result depends only on the seed."""
+    n = math.prod(shape)
+    out = torch.empty(n, dtype=torch.float32)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = torch.randn(e - s, generator=gen, dtype=torch.float32)
+    return out.view(*shape)
+
+
+def randn_bf16(shape, gen: torch.Generator) -> torch.Tensor:
+    """bf16 N(0,1): fp32 draws rounded to nearest-even, chunk by chunk."""
+    n = math.prod(shape)
+    out = torch.empty(n, dtype=torch.bfloat16)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = torch.randn(e - s, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+    return out.view(*shape)
+
+
+def uniform_lengths(n: int, lo: int, hi: int, gen: torch.Generator) -> list[int]:
+    """``n`` integers uniform on [lo, hi] inclusive."""
+    return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=gen)]
+
+
+def cu_seqlens_of(lengths) -> torch.Tensor:
+    """int32 [B+1] running totals of the lengths, starting at 0 (the varlen layout)."""
+    out = [0]
+    for L in lengths:
+        out.append(out[-1] + int(L))
+    return torch.tensor(out, dtype=torch.int32)
+
+
+def paged_layout(seq_lens, page_size: int, gen: torch.Generator):
+    """Scatter each request's pages over a pool by a seeded permutation.
+
+    The pool holds exactly sum(ceil(len/page_size)) pages.  Request b takes
+    the next ceil(len_b/page_size) entries of ``randperm(pool)``; unused
+    block-table entries are -1.  Returns (block_table int32 [B, max_blocks],
+    num_pages).
+    """
+    need = [(int(L) + page_size - 1) // page_size for L in seq_lens]
+    num_pages = sum(need)
+    max_blocks = max(need) if need else 0
+    perm = torch.randperm(num_pages, generator=gen).to(torch.int32)
+    bt = torch.full((len(need), max(max_blocks, 1)), -1, dtype=torch.int32)
+    off = 0
+    for b, n in enumerate(need):
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    return bt, num_pages
+
+
+@dataclass
+class PrefillInputs:
+    name: str
+    q: torch.Tensor            # [T, Hq, d] bf16
+    k: torch.Tensor            # [T, Hkv, d] bf16
+    v: torch.Tensor            # [T, Hkv, d] bf16
+    cu_seqlens: torch.Tensor   # [B+1] int32
+    lengths: list
+    causal: bool
+    scale: float               # the fp32 value both sides receive
+    q32: torch.Tensor | None = None   # fp32 originals (tiny workload only)
+    k32: torch.Tensor | None = None
+    v32: torch.Tensor | None = None
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def B(self):
+        return len(self.lengths)
+
+    @property
+    def Hq(self):
+        return self.q.shape[1]
+
+    @property
+    def Hkv(self):
+        return self.k.shape[1]
+
+    @property
+    def d(self):
+        return self.q.shape[2]
+
+    @property
+    def T(self):
+        return self.q.shape[0]
+
+
+@dataclass
+class DecodeInputs:
+    name: str
+    q: torch.Tensor            # [B, Hq, d] bf16
+    k_pages: torch.Tensor      # [num_pages, page_size, Hkv, d] bf16
+    v_pages: torch.Tensor
+    block_table: torch.Tensor  # [B, max_blocks] int32, -1 unused
+    seq_lens: torch.Tensor     # [B] int32
+    page_size: int
+    scale: float
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def B(self):
+        return self.q.shape[0]
+
+    @property
+    def Hq(self):
+        return self.q.shape[1]
+
+    @property
+    def Hkv(self):
+        return self.k_pages.shape[2]
+
+    @property
+    def d(self):
+        return self.q.shape[2]
+
+    @property
+    def num_pages(self):
+        return self.k_pages.shape[0]
+
+
+def fp32_scale(d: int) -> float:
+    """The default softmax scale 1/sqrt(head_dim), rounded once to fp32."""
+    return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32).item())
+
+
+def make_prefill(lengths, Hq: int, Hkv: int, d: int, causal: bool, seed: int,
+                 name: str = "prefill", keep_f32: bool = False,
+                 scale: float | None = None) -> PrefillInputs:
+    """Packed prefill inputs for the given sequence lengths."""
+    gen = torch.Generator().manual_seed(seed)
+    T = sum(int(L) for L in lengths)
+    if keep_f32:
+        q32 = randn_f32((T, Hq, d), gen)
+        k32 = randn_f32((T, Hkv, d), gen)
+        v32 = randn_f32((T, Hkv, d), gen)
+        q, k, v = (x.to(torch.bfloat16) for x in (q32, k32, v32))
+    else:
+        q32 = k32 = v32 = None
+        q = randn_bf16((T, Hq, d), gen)
+        k = randn_bf16((T, Hkv, d), gen)
+        v = randn_bf16((T, Hkv, d), gen)
+    return PrefillInputs(name=name, q=q, k=k, v=v, cu_seqlens=cu_seqlens_of(lengths),
+                         lengths=[int(L) for L in lengths], causal=causal,
+                         scale=fp32_scale(d) if scale is None else scale,
+                         q32=q32, k32=k32, v32=v32, meta={"seed": seed})
+
+
+def make_decode(seq_lens, Hq: int, Hkv: int, d: int, page_size: int, seed: int,
+                name: str = "decode", scale: float | None = None) -> DecodeInputs:
+    """Paged decode inputs for the given context lengths."""
+    gen = torch.Generator().manual_seed(seed)
+    bt, num_pages = paged_layout(seq_lens, page_size, gen)
+    B = len(seq_lens)
+    q = randn_bf16((B, Hq, d), gen)
+    k = randn_bf16((num_pages, page_size, Hkv, d), gen)
+    v = randn_bf16((num_pages, page_size, Hkv, d), gen)
+    return DecodeInputs(name=name, q=q, k_pages=k, v_pages=v, block_table=bt,
+                        seq_lens=torch.tensor([int(x) for x in seq_lens], dtype=torch.int32),
+                        page_size=page_size, scale=fp32_scale(d) if scale is None else scale,
+                        meta={"seed": seed})
+
+
+# ---------------------------------------------------------------------------
+# The five named workloads.  Seed 1000 + k for workload k.
+# ---------------------------------------------------------------------------
+
+WORKLOADS = {
+    "tiny": "B=1 H=1 L=256 d=64 fp32 N(0,1) with a bf16 copy, causal and non-causal",
+    "mha_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 bf16",
+    "varlen_gqa_prefill": "varlen GQA causal prefill, 8 seqs L~U[512,8192], Hq=32 Hkv=8 d=128",
+    "paged_decode": "paged decode, 64 requests, Hq=32 Hkv=8 d=128, ctx~U[1024,32768], page 16",
+    "long_decode": "split-KV decode, 2 requests x 131072 ctx, Hq=32 Hkv=8 d=128, page 64",
+}
+
+
+def tiny(causal: bool) -> PrefillInputs:
+    return make_prefill([256], 1, 1, 64, causal, seed=1001, name="tiny", keep_f32=True)
+
+
+def mha_prefill() -> PrefillInputs:
+    return make_prefill([2048] * 4, 16, 16, 128, True, seed=1002, name="mha_prefill")
+
+
+def varlen_gqa_prefill() -> PrefillInputs:
+    gen = torch.Generator().manual_seed(1003)
+    lengths = uniform_lengths(8, 512, 8192, gen)
+    T = sum(lengths)
+    q = randn_bf16((T, 32, 128), gen)
+    k = randn_bf16((T, 8, 128), gen)
+    v = randn_bf16((T, 8, 128), gen)
+    return PrefillInputs(name="varlen_gqa_prefill", q=q, k=k, v=v,
+                         cu_seqlens=cu_seqlens_of(lengths), lengths=lengths, causal=True,
+                         scale=fp32_scale(128), meta={"seed": 1003})
+
+
+def _decode_from_lengths(name, seq_lens, page_size, seed, gen):
+    bt, num_pages = paged_layout(seq_lens, page_size, gen)
+    B = len(seq_lens)
+    q = randn_bf16((B, 32, 128), gen)
+    k = randn_bf16((num_pages, page_size, 8, 128), gen)
+    v = randn_bf16((num_pages, page_size, 8, 128), gen)
+    return DecodeInputs(name=name, q=q, k_pages=k, v_pages=v, block_table=bt,
+                        seq_lens=torch.tensor(seq_lens, dtype=torch.int32),
+                        page_size=page_size, scale=fp32_scale(128), meta={"seed": seed})
+
+
+def paged_decode() -> DecodeInputs:
+    gen = torch.Generator().manual_seed(1004)
+    lens = uniform_lengths(64, 1024, 32768, gen)
+    return _decode_from_lengths("paged_decode", lens, 16, 1004, gen)
+
+
+def long_decode() -> DecodeInputs:
+    gen = torch.Generator().manual_seed(1005)
+    return _decode_from_lengths("long_decode", [131072, 131072], 64, 1005, gen)

@@ -1,0 +1,226 @@
+"""fp64 CPU oracle for exact attention (prefill and paged decode).
+
+TEST INFRASTRUCTURE ONLY.  The tests, the smoke check and the benchmark's
+CPU-baseline leg may import this package; the product path never does, and
+this package imports nothing from the product package.
+
+The arithmetic lives in ``oracle.c`` (plain definition, fp64, two-pass
+softmax over a materialised score row).  This module only marshals arrays
+into it: inputs may be torch CPU tensors or numpy arrays of bf16 (torch
+``bfloat16``), float32 or float64, and are passed to C in that element type
+so that the C code upcasts them exactly.
+
+Module-level functions use the library built from ``oracle.c``;
+``Oracle(path)`` binds any other build of the same source (the mutation
+tests use this to load copies with a planted mistake).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_BF16, _F32, _F64 = 0, 1, 2
+
+
+def _as_np(x):
+    """Return (numpy array, dtype code).  bf16 tensors become uint16 bit patterns."""
+    try:
+        import torch
+    except ImportError:  # pragma: no cover
+        torch = None
+    if torch is not None and isinstance(x, torch.Tensor):
+        x = x.detach().cpu().contiguous()
+        if x.dtype == torch.bfloat16:
+            return x.view(torch.int16).numpy().view(np.uint16), _BF16
+        if x.dtype == torch.float32:
+            return x.numpy(), _F32
+        if x.dtype == torch.float64:
+            return x.numpy(), _F64
+        raise TypeError(f"unsupported dtype {x.dtype}")
+    a = np.ascontiguousarray(x)
+    if a.dtype == np.float32:
+        return a, _F32
+    if a.dtype == np.float64:
+        return a, _F64
+    raise TypeError(f"unsupported dtype {a.dtype} (pass bf16 as a torch tensor)")
+
+
+def _int_np(x, dtype):
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x), dtype=dtype)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _same_dtype(*arrs):
+    codes = {c for _, c in arrs}
+    if len(codes) != 1:
+        raise TypeError("q, k and v must share one element type")
+    return codes.pop()
+
+
+class Oracle:
+    """ctypes binding of one build of ``oracle.c``."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        vp = ctypes.c_void_p
+        ci, cd, c64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
+        lib.oracle_prefill_rows.argtypes = [vp, vp, vp, ci, vp, ci, ci, ci, ci, ci, cd,
+                                            vp, vp, c64, vp, vp]
+        lib.oracle_prefill.argtypes = [vp, vp, vp, ci, vp, ci, ci, ci, ci, ci, cd, vp, vp]
+        lib.oracle_prefill_probs.argtypes = [vp, vp, ci, vp, ci, ci, ci, ci, ci, cd, ci, ci, vp]
+        lib.oracle_decode_paged.argtypes = [vp, vp, vp, ci, vp, vp, ci, ci, ci, ci, ci, ci,
+                                            c64, cd, vp, vp]
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_set_num_threads.argtypes = [ci]
+        for f in (lib.oracle_prefill_rows, lib.oracle_prefill, lib.oracle_prefill_probs,
+                  lib.oracle_decode_paged, lib.oracle_num_threads):
+            f.restype = ctypes.c_int
+        lib.oracle_set_num_threads.restype = None
+        self._lib = lib
+        self.path = path
+
+    def set_num_threads(self, n: int) -> None:
+        self._lib.oracle_set_num_threads(int(n))
+
+    def num_threads(self) -> int:
+        return int(self._lib.oracle_num_threads())
+
+    def prefill(self, q, k, v, cu_seqlens, causal: bool, scale: float):
+        """Exact attention over packed sequences.
+
+        q: [T, Hq, d]; k, v: [T, Hkv, d]; cu_seqlens: [B+1].
+        Returns (o [T, Hq, d] float64, lse [Hq, T] float64).
+        """
+        (qa, c1), (ka, c2), (va, c3) = _as_np(q), _as_np(k), _as_np(v)
+        dt = _same_dtype((qa, c1), (ka, c2), (va, c3))
+        cu = _int_np(cu_seqlens, np.int32)
+        T, Hq, d = qa.shape
+        Hkv = ka.shape[1]
+        B = cu.shape[0] - 1
+        o = np.zeros((T, Hq, d), np.float64)
+        lse = np.zeros((Hq, T), np.float64)
+        rc = self._lib.oracle_prefill(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(cu), B, Hq, Hkv,
+                                      d, int(bool(causal)), float(scale), _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError(f"oracle_prefill rejected its arguments (rc={rc})")
+        return o, lse
+
+    def prefill_rows(self, q, k, v, cu_seqlens, causal: bool, scale: float,
+                     rows_t: Sequence[int], rows_h: Sequence[int]):
+        """Exact attention for selected (token, head) rows only.
+
+        Returns (o [n, d] float64, lse [n] float64).  Rows are independent,
+        so a sample of rows is exact for those rows.
+        """
+        (qa, c1), (ka, c2), (va, c3) = _as_np(q), _as_np(k), _as_np(v)
+        dt = _same_dtype((qa, c1), (ka, c2), (va, c3))
+        cu = _int_np(cu_seqlens, np.int32)
+        rt = _int_np(rows_t, np.int64)
+        rh = _int_np(rows_h, np.int32)
+        T, Hq, d = qa.shape
+        Hkv = ka.shape[1]
+        B = cu.shape[0] - 1
+        n = rt.shape[0]
+        o = np.zeros((n, d), np.float64)
+        lse = np.zeros((n,), np.float64)
+        rc = self._lib.oracle_prefill_rows(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(cu), B, Hq,
+                                           Hkv, d, int(bool(causal)), float(scale), _ptr(rt),
+                                           _ptr(rh), n, _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError(f"oracle_prefill_rows rejected its arguments (rc={rc})")
+        return o, lse
+
+    def prefill_probs(self, q, k, cu_seqlens, causal: bool, scale: float, b: int, h: int,
+                      Hkv: int):
+        """The [L, L] probability matrix P of one (sequence, head); zeros where masked."""
+        (qa, c1), (ka, c2) = _as_np(q), _as_np(k)
+        dt = _same_dtype((qa, c1), (ka, c2))
+        cu = _int_np(cu_seqlens, np.int32)
+        T, Hq, d = qa.shape
+        B = cu.shape[0] - 1
+        L = int(cu[b + 1] - cu[b])
+        P = np.zeros((L, L), np.float64)
+        rc = self._lib.oracle_prefill_probs(_ptr(qa), _ptr(ka), dt, _ptr(cu), B, Hq, Hkv, d,
+                                            int(bool(causal)), float(scale), int(b), int(h),
+                                            _ptr(P))
+        if rc != 0:
+            raise ValueError(f"oracle_prefill_probs rejected its arguments (rc={rc})")
+        return P
+
+    def decode_paged(self, q, k_pages, v_pages, block_table, seq_lens, scale: float):
+        """Single-token attention of each request over its paged K/V cache.
+
+        q: [B, Hq, d]; k_pages, v_pages: [num_pages, page_size, Hkv, d];
+        block_table: [B, max_blocks] int32; seq_lens: [B] int32.
+        Returns (o [B, Hq, d] float64, lse [B, Hq] float64).
+        """
+        (qa, c1), (ka, c2), (va, c3) = _as_np(q), _as_np(k_pages), _as_np(v_pages)
+        dt = _same_dtype((qa, c1), (ka, c2), (va, c3))
+        bt = _int_np(block_table, np.int32)
+        sl = _int_np(seq_lens, np.int32)
+        B, Hq, d = qa.shape
+        num_pages, page_size, Hkv, _ = ka.shape
+        max_blocks = bt.shape[1]
+        o = np.zeros((B, Hq, d), np.float64)
+        lse = np.zeros((B, Hq), np.float64)
+        rc = self._lib.oracle_decode_paged(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(bt),
+                                           _ptr(sl), B, Hq, Hkv, d, page_size, max_blocks,
+                                           num_pages, float(scale), _ptr(o), _ptr(lse))
+        if rc == -2:
+            raise IndexError("a used block_table entry is outside [0, num_pages)")
+        if rc != 0:
+            raise ValueError(f"oracle_decode_paged rejected its arguments (rc={rc})")
+        return o, lse
+
+
+_default: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``oracle.c`` (built on first use).
+
+    ``ORACLE_LIB`` names another build of the same source instead; the
+    mutation tests point it at copies with a planted mistake.
+    """
+    global _default
+    if _default is None:
+        import os
+        _default = Oracle(os.environ.get("ORACLE_LIB") or _build.ensure_built())
+    return _default
+
+
+def prefill(*args, **kw):
+    return default().prefill(*args, **kw)
+
+
+def prefill_rows(*args, **kw):
+    return default().prefill_rows(*args, **kw)
+
+
+def prefill_probs(*args, **kw):
+    return default().prefill_probs(*args, **kw)
+
+
+def decode_paged(*args, **kw):
+    return default().decode_paged(*args, **kw)
+
+
+def set_num_threads(n: int) -> None:
+    default().set_num_threads(n)
+
+
+def num_threads() -> int:
+    return default().num_threads()

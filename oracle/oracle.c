@@ -1,0 +1,353 @@
+/*
+ * Exact-attention oracle: a plain, slow, fp64 CPU restatement of what the
+ * attention forward pass computes.  TEST INFRASTRUCTURE ONLY: the tests, the
+ * smoke check and the benchmark's CPU-baseline leg may load it; the product
+ * path never does.  It shares no code, header or constant with the CUDA
+ * library.
+ *
+ * What it follows (page, section):
+ *  - "FlashAttention-3 vs naive attention" (cnblogs), section 1.1: the basic
+ *    attention S = QK^T/sqrt(d) + mask, P = softmax(S), O = PV.  This file
+ *    writes that definition out literally, one query row at a time: all
+ *    scores of the row are materialised, the softmax is taken in two passes
+ *    (row max, then exponentials and their sum), and the output is the
+ *    P-weighted sum of V rows.  No tiling and no online recurrence: the pages
+ *    state that the tiled method is exactly equal to this (gsyq.cn FA vs FIA,
+ *    section 1; cnblogs section 1 and section 9).
+ *  - "flash-attention" skill page (skillsmp), section 3.2: causal mask and
+ *    the default softmax_scale = 1/sqrt(headdim); section 3.4: packed
+ *    variable-length batches described by cu_seqlens, with no attention
+ *    across sequences; appendix "GQA/MQA": q heads share kv heads without a
+ *    manual repeat (read as contiguous groups, kv head = h / (Hq/Hkv));
+ *    appendix "PagedAttention": a paged K/V pool [num_blocks, block_size,
+ *    kv_heads, head_dim] addressed through block_table[batch, max_blocks]
+ *    and cache_seqlens[batch], with one query token per request at the last
+ *    position (it sees every cached token).
+ *  - The log-sum-exp of each row (natural log, of the scaled logits) is
+ *    returned beside O; the pages name the row max m and sum l, and
+ *    LSE = m + ln l.
+ *
+ * Precision: every product and sum is in double.  Inputs are read in the
+ * caller's element type (bf16 bit patterns, fp32 or fp64) and upcast
+ * exactly.  The scale is taken as given (callers pass the fp32 value the GPU
+ * receives).
+ *
+ * Threading: OpenMP over independent (row, head) units only; each unit is
+ * computed by one thread in a fixed order, so results do not depend on the
+ * thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_BF16 = 0, OR_F32 = 1, OR_F64 = 2 };
+
+/* Exact upcast of one element of an input tensor. */
+static double elem(const void *base, size_t i, int dtype)
+{
+    if (dtype == OR_BF16) {
+        uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    if (dtype == OR_F32)
+        return (double)((const float *)base)[i];
+    return ((const double *)base)[i];
+}
+
+/*
+ * One query row against an explicit list of key/value rows.
+ *   qrow: element offset of the query vector (d consecutive elements)
+ *   krows/vrows: element offsets of each visible key/value vector
+ *   n: number of visible keys (n == 0 gives O = 0, LSE = -inf)
+ * s and p are caller scratch of length >= n.
+ */
+static void attend_one_row(const void *q, const void *k, const void *v, int dtype,
+                           size_t qrow, const size_t *krows, const size_t *vrows,
+                           size_t n, int d, double scale, double *s, double *p,
+                           double *o_out, double *lse_out)
+{
+    if (n == 0) {
+        for (int c = 0; c < d; ++c)
+            o_out[c] = 0.0;
+        *lse_out = -INFINITY;
+        return;
+    }
+    /* S_j = scale * <q, k_j> */
+    for (size_t j = 0; j < n; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c)
+            dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);
+        s[j] = scale * dot;
+    }
+    /* softmax, pass 1: the row max */
+    double m = s[0];
+    for (size_t j = 1; j < n; ++j)
+        if (s[j] > m)
+            m = s[j];
+    /* pass 2: exponentials, their sum, and the normalised probabilities */
+    double z = 0.0;
+    for (size_t j = 0; j < n; ++j) {
+        p[j] = exp(s[j] - m);
+        z += p[j];
+    }
+    for (size_t j = 0; j < n; ++j)
+        p[j] = p[j] / z;
+    /* O = sum_j P_j v_j */
+    for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (size_t j = 0; j < n; ++j)
+            acc += p[j] * elem(v, vrows[j] + (size_t)c, dtype);
+        o_out[c] = acc;
+    }
+    *lse_out = m + log(z);
+}
+
+/* Sequence index b such that cu[b] <= t < cu[b+1]; -1 if none. */
+static int seq_of_token(const int32_t *cu, int B, int64_t t)
+{
+    for (int b = 0; b < B; ++b)
+        if (t >= cu[b] && t < cu[b + 1])
+            return b;
+    return -1;
+}
+
+/*
+ * Prefill for an explicit list of (token, head) rows.
+ *   q: [T, Hq, d]; k, v: [T, Hkv, d]; cu_seqlens: [B+1] prefix sums.
+ *   rows_t/rows_h: the requested rows (nrows of them).
+ *   o: [nrows, d] (double); lse: [nrows] (double).
+ * Query token t of sequence b (local index i = t - cu[b]) sees keys
+ * cu[b] + j for j in [0, L_b) (non-causal) or j in [0, i] (causal).
+ * Returns 0, or -1 on an invalid argument.
+ */
+int oracle_prefill_rows(const void *q, const void *k, const void *v, int dtype,
+                        const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d,
+                        int causal, double scale, const int64_t *rows_t,
+                        const int32_t *rows_h, int64_t nrows, double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0)
+        return -1;
+    int64_t T = cu_seqlens[B];
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b) {
+        if (cu_seqlens[b + 1] < cu_seqlens[b])
+            return -1;
+        if (cu_seqlens[b + 1] - cu_seqlens[b] > maxlen)
+            maxlen = cu_seqlens[b + 1] - cu_seqlens[b];
+    }
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows_t[r] < 0 || rows_t[r] >= T || rows_h[r] < 0 || rows_h[r] >= Hq)
+            return -1;
+    const int group = Hq / Hkv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t cap = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *s = (double *)malloc(cap * sizeof(double));
+        double *p = (double *)malloc(cap * sizeof(double));
+        size_t *kr = (size_t *)malloc(cap * sizeof(size_t));
+        size_t *vr = (size_t *)malloc(cap * sizeof(size_t));
+        if (!s || !p || !kr || !vr) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nrows; ++r) {
+                int64_t t = rows_t[r];
+                int h = rows_h[r];
+                int kh = h / group;
+                int b = seq_of_token(cu_seqlens, B, t);
+                int64_t start = cu_seqlens[b];
+                int64_t L = cu_seqlens[b + 1] - start;
+                int64_t i = t - start;
+                int64_t n = causal ? i + 1 : L;
+                for (int64_t j = 0; j < n; ++j) {
+                    kr[j] = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;
+                    vr[j] = kr[j];
+                }
+                size_t qrow = ((size_t)t * (size_t)Hq + (size_t)h) * (size_t)d;
+                attend_one_row(q, k, v, dtype, qrow, kr, vr, (size_t)n, d, scale, s, p,
+                               o + (size_t)r * (size_t)d, lse + r);
+            }
+        }
+        free(s);
+        free(p);
+        free(kr);
+        free(vr);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Full prefill: every (token, head).  o: [T, Hq, d] double; lse: [Hq, T]
+ * double (may be NULL).
+ */
+int oracle_prefill(const void *q, const void *k, const void *v, int dtype,
+                   const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                   double scale, double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0)
+        return -1;
+    int64_t T = cu_seqlens[B];
+    int64_t nrows = T * Hq;
+    int64_t *rt = (int64_t *)malloc((size_t)(nrows > 0 ? nrows : 1) * sizeof(int64_t));
+    int32_t *rh = (int32_t *)malloc((size_t)(nrows > 0 ? nrows : 1) * sizeof(int32_t));
+    double *l = (double *)malloc((size_t)(nrows > 0 ? nrows : 1) * sizeof(double));
+    if (!rt || !rh || !l) {
+        free(rt);
+        free(rh);
+        free(l);
+        return -1;
+    }
+    /* row r = t*Hq + h, so o comes out directly in [T, Hq, d] order */
+    for (int64_t t = 0; t < T; ++t)
+        for (int h = 0; h < Hq; ++h) {
+            rt[t * Hq + h] = t;
+            rh[t * Hq + h] = h;
+        }
+    int rc = oracle_prefill_rows(q, k, v, dtype, cu_seqlens, B, Hq, Hkv, d, causal, scale,
+                                 rt, rh, nrows, o, l);
+    if (rc == 0 && lse)
+        for (int64_t t = 0; t < T; ++t)
+            for (int h = 0; h < Hq; ++h)
+                lse[(size_t)h * (size_t)T + (size_t)t] = l[t * Hq + h];
+    free(rt);
+    free(rh);
+    free(l);
+    return rc;
+}
+
+/*
+ * The probability matrix P of one (sequence, head) for small cases:
+ * P: [L, L] double, row i = query i, column j = key j, zero where masked.
+ */
+int oracle_prefill_probs(const void *q, const void *k, int dtype, const int32_t *cu_seqlens,
+                         int B, int Hq, int Hkv, int d, int causal, double scale, int b,
+                         int h, double *P)
+{
+    if (b < 0 || b >= B || h < 0 || h >= Hq || Hq % Hkv != 0)
+        return -1;
+    int64_t start = cu_seqlens[b];
+    int64_t L = cu_seqlens[b + 1] - start;
+    int kh = h / (Hq / Hkv);
+    double *s = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+    if (!s)
+        return -1;
+    for (int64_t i = 0; i < L; ++i) {
+        int64_t n = causal ? i + 1 : L;
+        size_t qrow = ((size_t)(start + i) * (size_t)Hq + (size_t)h) * (size_t)d;
+        for (int64_t j = 0; j < n; ++j) {
+            size_t krow = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c)
+                dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krow + (size_t)c, dtype);
+            s[j] = scale * dot;
+        }
+        double m = s[0];
+        for (int64_t j = 1; j < n; ++j)
+            if (s[j] > m)
+                m = s[j];
+        double z = 0.0;
+        for (int64_t j = 0; j < n; ++j)
+            z += exp(s[j] - m);
+        for (int64_t j = 0; j < L; ++j)
+            P[(size_t)i * (size_t)L + (size_t)j] = (j < n) ? exp(s[j] - m) / z : 0.0;
+    }
+    free(s);
+    return 0;
+}
+
+/*
+ * Paged decode: one query token per request at the last position.
+ *   q: [B, Hq, d]; k_pages, v_pages: [num_pages, page_size, Hkv, d]
+ *   block_table: [B, max_blocks] int32; seq_lens: [B] int32
+ *   o: [B, Hq, d] double; lse: [B, Hq] double (may be NULL)
+ * Token t of request b lives in page block_table[b][t / page_size], slot
+ * t % page_size.  Computed in one pass over all seq_len tokens, with no
+ * split: splitting is what the GPU path does and is checked against this.
+ * Returns 0, -1 on an invalid argument, -2 if a used block_table entry is
+ * outside [0, num_pages).
+ */
+int oracle_decode_paged(const void *q, const void *k_pages, const void *v_pages, int dtype,
+                        const int32_t *block_table, const int32_t *seq_lens, int B, int Hq,
+                        int Hkv, int d, int page_size, int max_blocks, int64_t num_pages,
+                        double scale, double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || page_size <= 0)
+        return -1;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b) {
+        if (seq_lens[b] < 0 || (int64_t)seq_lens[b] > (int64_t)max_blocks * page_size)
+            return -1;
+        if (seq_lens[b] > maxlen)
+            maxlen = seq_lens[b];
+        int64_t used = ((int64_t)seq_lens[b] + page_size - 1) / page_size;
+        for (int64_t i = 0; i < used; ++i) {
+            int32_t pg = block_table[(size_t)b * (size_t)max_blocks + (size_t)i];
+            if (pg < 0 || pg >= num_pages)
+                return -2;
+        }
+    }
+    const int group = Hq / Hkv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t cap = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *s = (double *)malloc(cap * sizeof(double));
+        double *p = (double *)malloc(cap * sizeof(double));
+        size_t *kr = (size_t *)malloc(cap * sizeof(size_t));
+        if (!s || !p || !kr) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < (int64_t)B * Hq; ++r) {
+                int b = (int)(r / Hq);
+                int h = (int)(r % Hq);
+                int kh = h / group;
+                int64_t n = seq_lens[b];
+                for (int64_t t = 0; t < n; ++t) {
+                    int64_t page = block_table[(size_t)b * (size_t)max_blocks + (size_t)(t / page_size)];
+                    int64_t slot = t % page_size;
+                    kr[t] = (((size_t)page * (size_t)page_size + (size_t)slot) * (size_t)Hkv +
+                             (size_t)kh) * (size_t)d;
+                }
+                double l;
+                attend_one_row(q, k_pages, v_pages, dtype, (size_t)r * (size_t)d, kr, kr,
+                               (size_t)n, d, scale, s, p, o + (size_t)r * (size_t)d, &l);
+                if (lse)
+                    lse[r] = l;
+            }
+        }
+        free(s);
+        free(p);
+        free(kr);
+    }
+    return bad ? -1 : 0;
+}
+
+/* Threads the OpenMP runtime will use (for reporting). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -1,0 +1,60 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case copies ``oracle/oracle.c``, plants one mistake of the kind a
+restatement of the definition could contain (a dropped term, a wrong sign,
+index or operand, an off-by-one mask, a wrong page address), builds it, and
+runs the pin suite against that build.  The suite must fail for every
+mutant; the unmodified source must pass it (``test_oracle_pins.py``).
+Everything runs on the CPU.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+from oracle import build as oracle_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+
+MUTANTS = {
+    "scale_dropped": ("s[j] = scale * dot;", "s[j] = dot;"),
+    "causal_excludes_diagonal": ("int64_t n = causal ? i + 1 : L;", "int64_t n = causal ? i : L;"),
+    "gqa_head_modulo": ("int kh = h / group;\n", "int kh = h % Hkv;\n"),
+    "lse_without_max": ("*lse_out = m + log(z);", "*lse_out = log(z);"),
+    "no_normalisation": ("p[j] = p[j] / z;", "p[j] = p[j];"),
+    "scores_use_values": ("dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);",
+                          "dot += elem(q, qrow + (size_t)c, dtype) * elem(v, krows[j] + (size_t)c, dtype);"),
+    "exp_sign_flipped": ("p[j] = exp(s[j] - m);", "p[j] = exp(m - s[j]);"),
+    "wrong_query_head": ("size_t qrow = ((size_t)t * (size_t)Hq + (size_t)h) * (size_t)d;",
+                         "size_t qrow = ((size_t)t * (size_t)Hq + (size_t)(Hq - 1 - h)) * (size_t)d;"),
+    "page_slot_wrong": ("int64_t slot = t % page_size;", "int64_t slot = (t / page_size) % page_size;"),
+    "decode_drops_last_token": ("int64_t n = seq_lens[b];", "int64_t n = seq_lens[b] - (seq_lens[b] > 1);"),
+    "values_reversed": ("acc += p[j] * elem(v, vrows[j] + (size_t)c, dtype);",
+                        "acc += p[j] * elem(v, vrows[n - 1 - j] + (size_t)c, dtype);"),
+    "keys_ignore_sequence_start": ("kr[j] = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;",
+                                   "kr[j] = ((size_t)(j) * (size_t)Hkv + (size_t)kh) * (size_t)d;"),
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle_build.SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    # the first occurrence is the main path (attend_one_row / prefill_rows come
+    # first in the file; oracle_prefill_probs repeats some lines further down)
+    assert source.count(old) >= 1, f"mutation site for {name} not found"
+    src = tmp_path / "oracle_mutant.c"
+    src.write_text(source.replace(old, new, 1))
+    lib = oracle_build.compile_oracle(str(src), str(tmp_path / "liboracle_mutant.so"))
+    env = dict(os.environ, ORACLE_LIB=lib, OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", PINS],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins accepted mutant {name}:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout, r.stdout[-2000:]
