@@ -1,0 +1,584 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one causal MHA prefill (B=4, Hq=Hkv=16, L=2048, d=128, bf16,
+O + LSE) followed by one paged decode (64 requests, Hq=32, Hkv=8, d=128,
+contexts U[1024, 32768] in 16-token pages, split-KV + LSE combine), both
+through the C ABI on inputs already resident in HBM.  Each kernel call is
+timed with CUDA events on the stream it is launched on; a 256 MB buffer is
+written between steps so the prefill inputs (100 MB) never start in L2 (the
+decode's 4.4 GB KV cache exceeds L2 anyway).
+
+Printed (rank 0, one JSON line): ``value`` = prefill TFLOP/s (causal pairs
+only, 4*d*Hq*L(L+1)/2 per sequence), with the decode's KV GB/s and both
+roofline fractions beside it; ``e2e`` repeats the measurement through the
+public API with pinned host buffers and the host<->device copies inside the
+timed region; ``cpu_baseline`` times the fp64 CPU oracle on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload step|...]
+    python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+Multi-GPU: launched by torch.distributed.run with one rank per GPU, every
+rank runs the same per-GPU workload (weak scaling, no data-path
+collective); the timed region is bracketed by barriers and the max over
+ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from exact_io_aware_86_b200 import api, inputs  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s (bf16) & paged-decode KV GB/s, % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, value: float, device=None) -> float:
+    """Max of a float over all ranks (identity on one rank)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# workload accounting
+# --------------------------------------------------------------------------
+def prefill_flops(lengths, Hq, d, causal=True) -> float:
+    pairs = sum(L * (L + 1) // 2 if causal else L * L for L in lengths)
+    return 4.0 * d * Hq * pairs
+
+
+def decode_bytes(inp) -> float:
+    """Algorithmic bytes of one decode call: K and V of every context token,
+    q and o, the used block-table entries and seq_lens."""
+    ctx = [int(x) for x in inp.seq_lens]
+    kv = sum(ctx) * inp.Hkv * inp.d * 2 * 2
+    qo = 2 * inp.B * inp.Hq * inp.d * 2
+    pages = sum((c + inp.page_size - 1) // inp.page_size for c in ctx)
+    return float(kv + qo + 4 * pages + 4 * inp.B)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(kind: str) -> str:
+    files = {"prefill": ["prefill_sm100.cuh", "ptx.cuh"], "decode": ["decode_sm100.cuh", "ptx.cuh"]}[kind]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "exact_io_aware_86_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kind: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None if the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(f"{kind}:{workload}")
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash(kind):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self._t is not None:
+                self._t.join(timeout=2)
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------
+# the oracle on a bounded sample (CPU baseline and reference arm)
+# --------------------------------------------------------------------------
+def oracle_prefill_sample(pin, n_pairs: int):
+    """Times the fp64 oracle on all rows of the first n_pairs (sequence, head)
+    pairs.  Returns (flops, seconds)."""
+    import numpy as np
+
+    import oracle
+    L = pin.lengths[0]
+    rt, rh, flops = [], [], 0.0
+    pairs = [(b, h) for b in range(pin.B) for h in range(pin.Hq)][:n_pairs]
+    for b, h in pairs:
+        start = int(pin.cu_seqlens[b])
+        rt.extend(range(start, start + L))
+        rh.extend([h] * L)
+        flops += prefill_flops([L], 1, pin.d, pin.causal)
+    t0 = time.perf_counter()
+    oracle.prefill_rows(pin.q, pin.k, pin.v, pin.cu_seqlens, pin.causal, pin.scale,
+                        np.array(rt), np.array(rh))
+    return flops, time.perf_counter() - t0
+
+
+def oracle_decode_sample(din, n_req: int):
+    """Times the fp64 oracle on the first n_req requests (all heads).
+    Returns (algorithmic bytes of those requests, seconds)."""
+    import oracle
+    sub = inputs.DecodeInputs("sample", din.q[:n_req], din.k_pages, din.v_pages,
+                              din.block_table[:n_req], din.seq_lens[:n_req], din.page_size,
+                              din.scale)
+    t0 = time.perf_counter()
+    oracle.decode_paged(sub.q, sub.k_pages, sub.v_pages, sub.block_table, sub.seq_lens, sub.scale)
+    return decode_bytes(sub), time.perf_counter() - t0
+
+
+def cpu_baseline(pin, din, budget_s: float = 20.0):
+    import oracle
+    cores = oracle.num_threads()
+    out = {"kind": "oracle", "cores": cores}
+    if pin is not None:
+        fl, sec = oracle_prefill_sample(pin, 1)
+        n = max(1, min(pin.B * pin.Hq, int((budget_s / 2) / max(sec, 1e-3))))
+        if n > 1:
+            fl, sec = oracle_prefill_sample(pin, n)
+        out.update(value=fl / sec / 1e12, unit="TFLOP/s",
+                   sample=f"all rows of {n} of {pin.B * pin.Hq} (sequence, head) pairs of {pin.name}")
+    if din is not None:
+        by, sec = oracle_decode_sample(din, 1)
+        n = max(1, min(din.B, int((budget_s / 2) / max(sec, 1e-3))))
+        if n > 1:
+            by, sec = oracle_decode_sample(din, n)
+        dec = {"value": by / sec / 1e9, "unit": "GB/s",
+               "sample": f"{n} of {din.B} requests (all heads) of {din.name}"}
+        if pin is None:
+            out.update(dec)
+        else:
+            out["decode"] = dec
+    return out
+
+
+# --------------------------------------------------------------------------
+# GPU measurement
+# --------------------------------------------------------------------------
+WORKLOAD_NAMES = {
+    "step": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 + paged decode 64 req Hq=32 Hkv=8 "
+            "d=128 ctx U[1024,32768] page 16",
+    "mha_prefill": inputs.WORKLOADS["mha_prefill"],
+    "varlen_gqa_prefill": inputs.WORKLOADS["varlen_gqa_prefill"],
+    "paged_decode": inputs.WORKLOADS["paged_decode"],
+    "long_decode": inputs.WORKLOADS["long_decode"],
+}
+
+
+def make_workload(name):
+    pin = din = None
+    if name in ("step", "mha_prefill"):
+        pin = inputs.mha_prefill()
+    if name == "varlen_gqa_prefill":
+        pin = inputs.varlen_gqa_prefill()
+    if name in ("step", "paged_decode"):
+        din = inputs.paged_decode()
+    if name == "long_decode":
+        din = inputs.long_decode()
+    return pin, din
+
+
+class DeviceWorkload:
+    """Device-resident inputs, outputs and scratch for the timed loop."""
+
+    def __init__(self, pin, din, dev):
+        self.pin, self.din = pin, din
+        if pin is not None:
+            self.q, self.k, self.v = (t.to(dev) for t in (pin.q, pin.k, pin.v))
+            self.cu = pin.cu_seqlens.to(dev)
+            self.o = torch.empty_like(self.q)
+            self.lse = torch.empty(pin.Hq, pin.T, dtype=torch.float32, device=dev)
+            self.max_len = max(pin.lengths)
+        if din is not None:
+            self.dq, self.kp, self.vp = (t.to(dev) for t in (din.q, din.k_pages, din.v_pages))
+            self.bt, self.sl = din.block_table.to(dev), din.seq_lens.to(dev)
+            self.splits = api.decode_auto_splits(din.B, din.Hkv, din.block_table.shape[1])
+            nbytes = api.decode_workspace_size(din.B, din.Hq, din.d, self.splits)
+            self.ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) if nbytes else None
+            self.do = torch.empty_like(self.dq)
+            self.dlse = torch.empty(din.B, din.Hq, dtype=torch.float32, device=dev)
+
+    def launches_per_step(self):
+        n = 1 if self.pin is not None else 0
+        if self.din is not None:
+            n += 1 + (1 if self.splits > 1 else 0)
+        return n
+
+    def prefill(self):
+        api.fa_prefill(self.q, self.k, self.v, self.o, self.lse, self.cu, self.pin.causal,
+                       self.pin.scale, self.max_len)
+
+    def decode(self):
+        api.fa_decode_paged(self.dq, self.kp, self.vp, self.bt, self.sl, self.splits, self.do,
+                            self.dlse, self.din.scale, self.ws)
+
+
+def time_device(w: DeviceWorkload, steps: int, warmup: int, dist, gpu_index: int):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        if w.pin is not None:
+            w.prefill()
+        if w.din is not None:
+            w.decode()
+    torch.cuda.synchronize()
+    if api.device_error() != api.FA_OK:
+        raise RuntimeError("device error during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(dist)
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_index) as clocks:
+        outer[0].record()
+        for i in range(steps):
+            flush.fill_(float(i))
+            ev[i][0].record()
+            if w.pin is not None:
+                w.prefill()
+            ev[i][1].record()
+            if w.din is not None:
+                w.decode()
+            ev[i][2].record()
+        outer[1].record()
+        torch.cuda.synchronize()
+        # keep sampling a little so short regions still get a sample
+        time.sleep(0.25)
+    barrier(dist)
+    pre = [ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)]
+    dec = [ev[i][1].elapsed_time(ev[i][2]) for i in range(steps)]
+    region = outer[0].elapsed_time(outer[1])
+    if api.device_error() != api.FA_OK:
+        raise RuntimeError("device error during the timed loop")
+    return pre, dec, region, clocks.summary()
+
+
+def time_e2e(w: DeviceWorkload, steps: int):
+    """Same step through the public API with pinned host inputs: H2D of the
+    step's inputs, the kernels, D2H of the results, all inside the timed
+    region.  Returns (prefill ms list, decode ms list, h2d bytes, d2h bytes)."""
+    pin, din = w.pin, w.din
+    host, h2d, d2h = {}, 0, 0
+    if pin is not None:
+        for n, t in (("q", pin.q), ("k", pin.k), ("v", pin.v), ("cu", pin.cu_seqlens)):
+            host[n] = t.pin_memory()
+            h2d += t.numel() * t.element_size()
+        host["o"] = torch.empty(w.o.shape, dtype=w.o.dtype, pin_memory=True)
+        host["lse"] = torch.empty(w.lse.shape, dtype=w.lse.dtype, pin_memory=True)
+        d2h += w.o.numel() * 2 + w.lse.numel() * 4
+    if din is not None:
+        for n, t in (("dq", din.q), ("kp", din.k_pages), ("vp", din.v_pages),
+                     ("bt", din.block_table), ("sl", din.seq_lens)):
+            host[n] = t.pin_memory()
+            h2d += t.numel() * t.element_size()
+        host["do"] = torch.empty(w.do.shape, dtype=w.do.dtype, pin_memory=True)
+        host["dlse"] = torch.empty(w.dlse.shape, dtype=w.dlse.dtype, pin_memory=True)
+        d2h += w.do.numel() * 2 + w.dlse.numel() * 4
+    pre, dec = [], []
+    for i in range(steps + 1):  # first iteration is a warm-up
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        if pin is not None:
+            w.q.copy_(host["q"], non_blocking=True)
+            w.k.copy_(host["k"], non_blocking=True)
+            w.v.copy_(host["v"], non_blocking=True)
+            w.cu.copy_(host["cu"], non_blocking=True)
+            w.prefill()
+            host["o"].copy_(w.o, non_blocking=True)
+            host["lse"].copy_(w.lse, non_blocking=True)
+        e[1].record()
+        if din is not None:
+            w.dq.copy_(host["dq"], non_blocking=True)
+            w.kp.copy_(host["kp"], non_blocking=True)
+            w.vp.copy_(host["vp"], non_blocking=True)
+            w.bt.copy_(host["bt"], non_blocking=True)
+            w.sl.copy_(host["sl"], non_blocking=True)
+            w.decode()
+            host["do"].copy_(w.do, non_blocking=True)
+            host["dlse"].copy_(w.dlse, non_blocking=True)
+        e[2].record()
+        torch.cuda.synchronize()
+        if i > 0:
+            pre.append(e[0].elapsed_time(e[1]))
+            dec.append(e[1].elapsed_time(e[2]))
+    return pre, dec, h2d, d2h
+
+
+def roofline(kind, achieved, peak, unit, traffic):
+    return {"bound": "tensor" if kind == "prefill" else "hbm", "achieved": round(achieved, 2),
+            "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic}
+
+
+def run_gpu(args, world, rank, local):
+    torch.cuda.set_device(local)
+    dist = init_dist(world, "nccl")
+    threads = max(1, (os.cpu_count() or 8) // max(world, 1))
+    torch.set_num_threads(threads)
+    pin, din = make_workload(args.workload)
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(pin, din, budget_s=args.cpu_budget)
+    w = DeviceWorkload(pin, din, torch.device("cuda", local))
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit() else local
+    pre, dec, region, clocks = time_device(w, args.steps, args.warmup, dist, gpu_index)
+    e2e_steps = max(2, min(args.steps, args.e2e_steps))
+    epre, edec, h2d, d2h = time_e2e(w, e2e_steps)
+
+    peaks, peak_src = load_peaks()
+    pre_ms = max_over_ranks(dist, statistics.mean(pre) if pin is not None else 0.0, "cuda")
+    dec_ms = max_over_ranks(dist, statistics.mean(dec) if din is not None else 0.0, "cuda")
+    reg_ms = max_over_ranks(dist, region, "cuda")
+    epre_ms = max_over_ranks(dist, statistics.mean(epre) if pin is not None else 0.0, "cuda")
+    edec_ms = max_over_ranks(dist, statistics.mean(edec) if din is not None else 0.0, "cuda")
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    parts, line = {}, {}
+    if pin is not None:
+        fl = prefill_flops(pin.lengths, pin.Hq, pin.d, pin.causal)
+        tf = world * fl / (pre_ms * 1e-3) / 1e12
+        parts["prefill"] = {
+            "workload": pin.name, "value": round(tf, 2), "unit": "TFLOP/s",
+            "ms": round(pre_ms, 4), "ms_min": round(min(pre), 4), "flops": fl,
+            "roofline": roofline("prefill", tf / world, peaks["bf16_tflops"], "TFLOP/s",
+                                 dram_traffic("prefill", pin.name)),
+            "launches_per_call": 1,
+        }
+    if din is not None:
+        by = decode_bytes(din)
+        gbs = world * by / (dec_ms * 1e-3) / 1e9
+        parts["decode"] = {
+            "workload": din.name, "value": round(gbs, 1), "unit": "GB/s",
+            "ms": round(dec_ms, 4), "ms_min": round(min(dec), 4), "bytes": by,
+            "num_splits": w.splits,
+            "workspace_bytes": api.decode_workspace_size(din.B, din.Hq, din.d, w.splits),
+            "roofline": roofline("decode", gbs / world, peaks["hbm_gbs"], "GB/s",
+                                 dram_traffic("decode", din.name)),
+            "launches_per_call": 1 + (1 if w.splits > 1 else 0),
+        }
+    head = parts.get("prefill") or parts.get("decode")
+    dominant = max(parts.values(), key=lambda p: p["ms"])
+    e2e = {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if pin is not None:
+        e2e.update(value=round(world * parts["prefill"]["flops"] / (epre_ms * 1e-3) / 1e12, 3),
+                   unit="TFLOP/s", ms=round(epre_ms, 3))
+    if din is not None:
+        dv = {"value": round(world * parts["decode"]["bytes"] / (edec_ms * 1e-3) / 1e9, 2),
+              "unit": "GB/s", "ms": round(edec_ms, 3)}
+        if pin is None:
+            e2e.update(dv)
+        else:
+            e2e["decode"] = dv
+    line = {
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": head["unit"],
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(pre_ms + dec_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[args.workload],
+                   "l2": "256 MB buffer written between steps; decode KV (4.4 GB) exceeds L2",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "parts": parts,
+        "roofline": dict(dominant["roofline"], kernel=dominant["workload"]),
+        "peaks_source": peak_src,
+        "region_ms": round(reg_ms, 3),
+        "e2e": e2e,
+        "gpu_launches": w.launches_per_step() * args.steps,
+        "clocks": clocks,
+    }
+    if base is not None:
+        line["cpu_baseline"] = base
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle, timed on the host cores on a
+    bounded sample of the same workload; same metric, unit and config."""
+    if rank != 0:
+        return
+    import oracle
+    pin, din = make_workload(args.workload)
+    pairs = 1
+    reqs = 2
+    for _ in range(max(0, args.warmup)):
+        if pin is not None:
+            oracle_prefill_sample(pin, pairs)
+        if din is not None:
+            oracle_decode_sample(din, reqs)
+        break  # one warm-up pass is enough for a CPU code path
+    pf, ps, db, ds = 0.0, 0.0, 0.0, 0.0
+    for _ in range(args.steps):
+        if pin is not None:
+            f, s = oracle_prefill_sample(pin, pairs)
+            pf, ps = pf + f, ps + s
+        if din is not None:
+            b, s = oracle_decode_sample(din, reqs)
+            db, ds = db + b, ds + s
+    parts = {}
+    if pin is not None:
+        parts["prefill"] = {"workload": pin.name, "value": pf / ps / 1e12, "unit": "TFLOP/s",
+                            "ms": 1e3 * ps / args.steps}
+    if din is not None:
+        parts["decode"] = {"workload": din.name, "value": db / ds / 1e9, "unit": "GB/s",
+                           "ms": 1e3 * ds / args.steps}
+    head = parts.get("prefill") or parts.get("decode")
+    sample = []
+    if pin is not None:
+        sample.append(f"prefill: all rows of {pairs} of {pin.B * pin.Hq} (sequence, head) pairs")
+    if din is not None:
+        sample.append(f"decode: {reqs} of {din.B} requests, all heads")
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": head["unit"], "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(p["ms"] for p in parts.values()), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[args.workload],
+                   "l2": "n/a (CPU)", "parallelism": "host cores"},
+        "parts": parts,
+        "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "value": head["value"],
+                         "unit": head["unit"], "sample": "; ".join(sample)},
+        "e2e": {"value": head["value"], "unit": head["unit"], "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_NAMES), default="step")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

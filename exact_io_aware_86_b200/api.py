@@ -1,0 +1,232 @@
+"""Python binding of ``libfa.so`` (C ABI in ``include/fa.h``).
+
+Argument marshalling only: shapes, dtypes and device pointers of torch
+tensors are passed to the C entry points, which run every step of the
+computation in this package's CUDA kernels.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_CUDA = 3
+FA_ERR_DEVICE_BOUNDS = 4
+FA_ERR_DEVICE_TIMEOUT = 5
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    """A non-OK status from the C ABI."""
+
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {error_string(code)} (status {code})")
+
+
+def load_library(path: str = LIB_PATH):
+    """Load ``libfa.so`` and declare its signatures (idempotent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing; build it with `python -m exact_io_aware_86_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, i32]
+    lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32, i32, i32,
+                                    i32, f32, vp, vp, sz]
+    lib.fa_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.fa_decode_workspace_size.restype = sz
+    lib.fa_decode_auto_splits.argtypes = [i32, i32, i32, i32]
+    lib.fa_prefill_f32.argtypes = lib.fa_prefill.argtypes
+    lib.fa_decode_paged_f32.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
+                                        i32, f32, vp]
+    lib.fa_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.fa_get_error_string.argtypes = [i32]
+    lib.fa_get_error_string.restype = ctypes.c_char_p
+    lib.fa_version.argtypes = []
+    for f in (lib.fa_prefill, lib.fa_decode_paged, lib.fa_decode_auto_splits, lib.fa_prefill_f32,
+              lib.fa_decode_paged_f32, lib.fa_get_device_error, lib.fa_version):
+        f.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def error_string(code: int) -> str:
+    return load_library().fa_get_error_string(int(code)).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != FA_OK:
+        raise FAError(code, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# --------------------------------------------------------------------------
+# prefill
+# --------------------------------------------------------------------------
+def fa_prefill(q, k, v, o, lse, cu_seqlens, causal: bool, scale: float = 0.0,
+               max_seqlen: int | None = None, stream=None, *, _f32: bool = False) -> None:
+    """Calls ``fa_prefill`` (bf16) or ``fa_prefill_f32`` on torch CUDA tensors.
+
+    q [T, Hq, d], k/v [T, Hkv, d], o [T, Hq, d], lse [Hq, T] fp32 or None,
+    cu_seqlens int32 [B+1].  ``max_seqlen`` bounds every sequence length
+    (defaults to T, which needs no device read).
+    """
+    dt = torch.float32 if _f32 else torch.bfloat16
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n, dt, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (T, Hkv, d) or v.shape != k.shape or o.shape != q.shape:
+        raise ValueError("q/k/v/o shapes disagree")
+    if lse is not None and lse.shape != (Hq, T):
+        raise ValueError("lse must be [Hq, T]")
+    B = cu_seqlens.numel() - 1
+    ms = T if max_seqlen is None else int(max_seqlen)
+    fn = load_library().fa_prefill_f32 if _f32 else load_library().fa_prefill
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), B, Hq, Hkv, d,
+              int(bool(causal)), float(scale), _stream(stream), T, ms),
+           "fa_prefill_f32" if _f32 else "fa_prefill")
+
+
+def prefill(q, k, v, cu_seqlens, causal: bool = True, scale: float = 0.0,
+            max_seqlen: int | None = None, return_lse: bool = True, stream=None):
+    """Allocates O (and LSE) and runs ``fa_prefill``.  Returns (o, lse or None)."""
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device) if return_lse else None
+    fa_prefill(q, k, v, o, lse, cu_seqlens, causal, scale, max_seqlen, stream)
+    return o, lse
+
+
+def prefill_f32(q, k, v, cu_seqlens, causal: bool = True, scale: float = 0.0, stream=None):
+    """fp32 debug path: returns (o fp32, lse fp32)."""
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device)
+    fa_prefill(q, k, v, o, lse, cu_seqlens, causal, scale, None, stream, _f32=True)
+    return o, lse
+
+
+# --------------------------------------------------------------------------
+# paged decode
+# --------------------------------------------------------------------------
+def decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:
+    return int(load_library().fa_decode_workspace_size(B, Hq, d, num_splits))
+
+
+def decode_auto_splits(B: int, Hkv: int, max_blocks_per_seq: int, num_sms: int = 0) -> int:
+    return int(load_library().fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, num_sms))
+
+
+def _decode_shapes(q, k_pages, v_pages, block_table, seq_lens, dt):
+    _need(q, "q", dt, 3)
+    _need(k_pages, "k_pages", dt, 4)
+    _need(v_pages, "v_pages", dt, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv, d2 = k_pages.shape
+    if d2 != d or v_pages.shape != k_pages.shape:
+        raise ValueError("q/k_pages/v_pages shapes disagree")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row per request")
+    return B, Hq, Hkv, d, num_pages, page_size, block_table.shape[1]
+
+
+def fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int, o, lse=None,
+                    scale: float = 0.0, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Calls ``fa_decode_paged`` on torch CUDA tensors.
+
+    q [B, Hq, d] bf16; k_pages/v_pages [num_pages, page_size, Hkv, d] bf16;
+    block_table [B, max_blocks] int32; seq_lens [B] int32; o [B, Hq, d] bf16;
+    lse [B, Hq] fp32 or None; workspace: a uint8 CUDA tensor of at least
+    ``decode_workspace_size`` bytes, or None (the library then allocates
+    stream-ordered scratch).
+    """
+    B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
+        q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16)
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    ws_bytes = 0
+    if workspace is not None:
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load_library().fa_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), page_size,
+        int(num_splits), _ptr(o), _stream(stream), B, Hq, Hkv, d, max_blocks, num_pages,
+        float(scale), _ptr(lse), _ptr(workspace), ws_bytes), "fa_decode_paged")
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int = 0,
+                 scale: float = 0.0, return_lse: bool = True, stream=None):
+    """Allocates O, LSE and the split workspace with torch and runs
+    ``fa_decode_paged``.  Returns (o, lse or None)."""
+    B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
+        q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16)
+    S = num_splits if num_splits > 0 else decode_auto_splits(B, Hkv, max_blocks)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if return_lse else None
+    nbytes = decode_workspace_size(B, Hq, d, S)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device) if nbytes else None
+    fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, S, o, lse, scale, ws, stream)
+    return o, lse
+
+
+def decode_paged_f32(q, k_pages, v_pages, block_table, seq_lens, scale: float = 0.0, stream=None):
+    """fp32 debug path: returns (o fp32, lse fp32)."""
+    B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
+        q, k_pages, v_pages, block_table, seq_lens, torch.float32)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    _check(load_library().fa_decode_paged_f32(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), page_size,
+        _ptr(o), _stream(stream), B, Hq, Hkv, d, max_blocks, num_pages, float(scale), _ptr(lse)),
+        "fa_decode_paged_f32")
+    return o, lse
+
+
+def device_error(stream=None) -> int:
+    """Reads and clears the device error word (synchronises the stream)."""
+    code = ctypes.c_int(0)
+    _check(load_library().fa_get_device_error(_stream(stream), ctypes.byref(code)),
+           "fa_get_device_error")
+    return code.value

@@ -1,0 +1,341 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: host-side argument checks,
+// TMA tensor maps, launch configuration, and the device error word.
+//
+// All kernels live in this one translation unit so they share the error
+// word (ptx.cuh) without relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "ptx.cuh"
+#include "prefill_sm100.cuh"
+#include "decode_sm100.cuh"
+#include "debug_f32.cuh"
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// --------------------------------------------------------------------------
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly (it loads on machines without a
+// GPU driver; the symbol is resolved on first use).
+// --------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first,
+// strides in bytes for dims 1.. (dim 0 is contiguous).
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms_current() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / sqrtf((float)d); }
+
+// Largest divisor of Hkv that is <= 8: kv heads handled by one decode CTA.
+int heads_per_cta(int Hkv) {
+  for (int h = fa::decode::MAX_HPB; h >= 1; --h)
+    if (Hkv % h == 0) return h;
+  return 1;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+template <int D>
+fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const int32_t* cu, int B, int Hq, int Hkv, int causal, float scale,
+                         cudaStream_t stream, int T, int max_seqlen) {
+  using namespace fa::prefill;
+  CUtensorMap tq, tk, tv;
+  const cuuint32_t box[2] = {64, (cuuint32_t)BM};
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)Hq * D, (cuuint64_t)T};
+    const cuuint64_t str[1] = {(cuuint64_t)Hq * D * 2};
+    if (!make_map(&tq, q, 2, dims, str, box)) return FA_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)Hkv * D, (cuuint64_t)T};
+    const cuuint64_t str[1] = {(cuuint64_t)Hkv * D * 2};
+    if (!make_map(&tk, k, 2, dims, str, box)) return FA_ERR_CUDA;
+    if (!make_map(&tv, v, 2, dims, str, box)) return FA_ERR_CUDA;
+  }
+  Params p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.cu_seqlens = cu;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.T = T;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = resolve_scale(scale, D) * kLog2e;
+  p.num_levels = (max_seqlen + ROWS_PER_ITEM - 1) / ROWS_PER_ITEM;
+
+  const int sms = num_sms_current();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long upper = ((long long)T / ROWS_PER_ITEM + B) * Hq;  // >= number of work items
+  long long grid = upper < sms ? upper : sms;
+  if (grid < 1) grid = 1;
+  if ((upper + grid - 1) / grid > MAX_ITEMS_PER_CTA) grid = (upper + MAX_ITEMS_PER_CTA - 1) / MAX_ITEMS_PER_CTA;
+  if (grid > 0x7fffffff) return FA_ERR_UNSUPPORTED;
+
+  const int smem = smem_bytes<D>();
+  static bool attr_ok = set_smem(prefill_kernel<D>, smem);
+  if (!attr_ok) return FA_ERR_CUDA;
+  prefill_kernel<D><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_decode(const void* q, const void* kp, const void* vp, const int32_t* bt,
+                        const int32_t* sl, int page_size, int S, void* o, cudaStream_t stream,
+                        int B, int Hq, int Hkv, int max_blocks, int num_pages, float scale,
+                        float* lse, void* ws) {
+  using namespace fa::decode;
+  const int hpb = heads_per_cta(Hkv);
+  CUtensorMap tk, tv;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv,
+                                (cuuint64_t)num_pages * (cuuint64_t)page_size};
+    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)TOK};
+    if (!make_map(&tk, kp, 3, dims, str, box)) return FA_ERR_CUDA;
+    if (!make_map(&tv, vp, 3, dims, str, box)) return FA_ERR_CUDA;
+  }
+  Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = bt;
+  p.seq_lens = sl;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.hpb = hpb;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks;
+  p.num_pages = num_pages;
+  p.num_splits = S;
+  p.half_bytes = Cfg<D>::PANELS * hpb * BOX_BYTES;
+  p.scale_log2 = resolve_scale(scale, D) * kLog2e;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  const size_t opart_bytes = round_up((size_t)B * Hq * S * D * sizeof(float), 256);
+  p.o_part = S > 1 ? static_cast<float*>(ws) : nullptr;
+  p.lse_part = S > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + opart_bytes) : nullptr;
+
+  const int smem = STAGES * stage_bytes(p.half_bytes) + 1024 + 64;
+  static bool attr_ok = set_smem(split_kernel<D>, STAGES * stage_bytes(Cfg<D>::PANELS * MAX_HPB * BOX_BYTES) + 1024 + 64);
+  if (!attr_ok) return FA_ERR_CUDA;
+  const dim3 grid((unsigned)S, (unsigned)(Hkv / hpb), (unsigned)B);
+  split_kernel<D><<<grid, (hpb + 1) * 32, smem, stream>>>(tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (S > 1) {
+    const int rows = B * Hq;
+    combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(p.o_part, p.lse_part, p.o, lse, rows, S);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const int32_t* cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                     float scale, fa_stream_t stream, int total_tokens, int max_seqlen) {
+  if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0 || max_seqlen < 0)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(cu_seqlens, 4) || (lse && !aligned(lse, 4)))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hq > 0xFFFF) return FA_ERR_UNSUPPORTED;
+  if ((long long)(max_seqlen + fa::prefill::ROWS_PER_ITEM - 1) / fa::prefill::ROWS_PER_ITEM >
+      fa::prefill::MAX_LEVELS)
+    return FA_ERR_UNSUPPORTED;
+  if (B == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_prefill<64>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
+                              total_tokens, max_seqlen);
+  return launch_prefill<128>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
+                             total_tokens, max_seqlen);
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || d <= 0 || num_splits <= 1) return 0;
+  const size_t o_part = round_up((size_t)B * Hq * num_splits * d * sizeof(float), 256);
+  const size_t l_part = round_up((size_t)B * Hq * num_splits * sizeof(float), 256);
+  return o_part + l_part;
+}
+
+int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int num_sms) {
+  if (B <= 0 || Hkv <= 0 || max_blocks_per_seq <= 0) return 1;
+  if (num_sms <= 0) num_sms = num_sms_current();
+  if (num_sms <= 0) num_sms = 148;
+  const long long units = (long long)B * (Hkv / heads_per_cta(Hkv));
+  const long long target = 4LL * num_sms;  // work units to spread over the SMs
+  long long s = (target + units - 1) / units;
+  if (s > max_blocks_per_seq) s = max_blocks_per_seq;
+  if (s > 1024) s = 1024;
+  if (s < 1) s = 1;
+  return (int)s;
+}
+
+fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                          const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                          int num_splits, void* o, fa_stream_t stream, int B, int Hq, int Hkv,
+                          int d, int max_blocks_per_seq, int num_pages, float scale, float* lse,
+                          void* workspace, size_t workspace_bytes) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || page_size < 1 || num_splits < 0 ||
+      max_blocks_per_seq < 1 || num_pages < 0)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(o, 16) ||
+      !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)) ||
+      (workspace && !aligned(workspace, 256)))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > fa::decode::MAX_GROUP) return FA_ERR_UNSUPPORTED;
+  if (page_size % fa::decode::TOK != 0) return FA_ERR_UNSUPPORTED;
+  if ((long long)num_pages * page_size > 0x7fffffffLL ||
+      (long long)max_blocks_per_seq * page_size > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv / heads_per_cta(Hkv) > 65535) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  const int S = num_splits == 0 ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, 0) : num_splits;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t need = fa_decode_workspace_size(B, Hq, d, S);
+  void* ws = workspace;
+  bool owned = false;
+  if (need > 0) {
+    if (ws) {
+      if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+    } else {
+      if (cudaMallocAsync(&ws, need, s) != cudaSuccess) return FA_ERR_CUDA;
+      owned = true;
+    }
+  }
+  fa_status st;
+  if (d == 64)
+    st = launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, page_size, S, o, s, B, Hq,
+                           Hkv, max_blocks_per_seq, num_pages, scale, lse, ws);
+  else
+    st = launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, page_size, S, o, s, B,
+                            Hq, Hkv, max_blocks_per_seq, num_pages, scale, lse, ws);
+  if (owned && cudaFreeAsync(ws, s) != cudaSuccess && st == FA_OK) st = FA_ERR_CUDA;
+  return st;
+}
+
+fa_status fa_prefill_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                         const int32_t* cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                         float scale, fa_stream_t stream, int total_tokens, int max_seqlen) {
+  (void)max_seqlen;
+  if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0 || d < 1)
+    return FA_ERR_INVALID_ARG;
+  if (d > fa::debug::MAX_D) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || total_tokens == 0) return FA_OK;
+  const long long n = (long long)total_tokens * Hq;
+  const long long blocks = (n + 127) / 128;
+  if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  fa::debug::prefill_f32_kernel<<<(unsigned)blocks, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, d, causal ? 1 : 0, resolve_scale(scale, d),
+      total_tokens);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_decode_paged_f32(const float* q, const float* k_pages, const float* v_pages,
+                              const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                              float* o, fa_stream_t stream, int B, int Hq, int Hkv, int d,
+                              int max_blocks_per_seq, int num_pages, float scale, float* lse) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || page_size < 1 || max_blocks_per_seq < 1 ||
+      num_pages < 0 || d < 1)
+    return FA_ERR_INVALID_ARG;
+  if (d > fa::debug::MAX_D) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  const long long n = (long long)B * Hq;
+  fa::debug::decode_f32_kernel<<<(unsigned)((n + 127) / 128), 128, 0,
+                                 reinterpret_cast<cudaStream_t>(stream)>>>(
+      q, k_pages, v_pages, block_table, seq_lens, page_size, o, lse, B, Hq, Hkv, d,
+      max_blocks_per_seq, num_pages, resolve_scale(scale, d));
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_get_device_error(fa_stream_t stream, int* code) {
+  if (!code) return FA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_device_error, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(fa::g_device_error, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v & fa::kDevErrTimeout) *code = FA_ERR_DEVICE_TIMEOUT;
+  else if (v & fa::kDevErrBounds) *code = FA_ERR_DEVICE_BOUNDS;
+  else *code = FA_OK;
+  return FA_OK;
+}
+
+const char* fa_get_error_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_CUDA: return "CUDA runtime or launch error";
+    case FA_ERR_DEVICE_BOUNDS: return "device-side index out of range";
+    case FA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,477 @@
+// prefill_sm100.cuh -- exact attention prefill on the 5th-generation tensor
+// cores (tcgen05), packed variable-length sequences, causal or full mask,
+// grouped kv heads.
+//
+// Method (pages: "gsyq.cn FA vs FIA" section 1, tiling + online softmax;
+// "FlashAttention" concept page, Tiling: Q in B_r-row blocks, K/V in
+// B_c-row blocks held on chip; cnblogs section 3.2 / 4.2: S and P never
+// written to HBM, QK^T + mask + softmax + PV fused in one kernel):
+//   for each 128-row query tile, stream 128-key K/V tiles; S = Q K_j^T on
+//   the tensor cores into tensor memory; the softmax warps read S, keep the
+//   running row max m and sum l, write P = exp(S*scale - m) back into tensor
+//   memory as bf16, and the tensor cores accumulate O += P V_j in tensor
+//   memory.  At the end O / l is stored as bf16 and LSE = ln2*(m + log2 l).
+//
+// CTA layout (320 threads, one CTA per SM, persistent):
+//   warp 0      TMA producer: Q tiles once per work item, then K_j, V_j
+//               alternately through a ring of 128 x D smem slots
+//   warp 1      MMA issuer (one thread) and TMEM owner (512 columns)
+//   warps 2-5   softmax for query tile 0 (rows q0 .. q0+127)
+//   warps 6-9   softmax for query tile 1 (rows q0+128 .. q0+255)
+// The two query tiles share every K/V tile, and while one softmax group
+// works on its S the tensor cores run the other tile's P V and Q K^T.
+//
+// Tensor memory columns: S0 [0,128), S1 [128,256), O0 [256,256+D),
+// O1 [384,384+D).  P_t (bf16, 2 per column) overwrites the first 64 columns
+// of S_t once S_t has been read; the MMA that writes the next S_t is issued
+// after the P_t V MMA, and tcgen05 MMAs from one thread execute in order.
+//
+// Lazy rescaling: a row's reference max m only moves when the tile max
+// exceeds it by more than 8 (log2 units), so P <= 256 and O is rescaled in
+// tensor memory only on those (rare) tiles.  The final O / l and the LSE use
+// the same reference max, so the result is exact up to rounding.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fa {
+namespace prefill {
+
+constexpr int BM = 128;           // query rows per tile
+constexpr int BN = 128;           // keys per K/V tile
+constexpr int NQT = 2;            // query tiles per work item
+constexpr int ROWS_PER_ITEM = NQT * BM;
+constexpr int NUM_WARPS = 10;
+constexpr int NUM_THREADS = NUM_WARPS * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr int MAX_LEVELS = 1024;  // max_seqlen <= 1024 * 256
+constexpr int MAX_ITEMS_PER_CTA = 256;
+
+template <int D>
+struct Cfg {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static constexpr int PANELS = D / 64;              // 64-element (128 B) swizzle panels
+  static constexpr int PANEL_BYTES = BM * 128;       // 128 rows x 128 B
+  static constexpr int TILE_BYTES = BM * D * 2;      // one Q, K or V tile
+  static constexpr int STAGES = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = NQT * TILE_BYTES;
+  static constexpr int SMEM_TILES = KV_OFF + STAGES * TILE_BYTES;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+};
+
+struct Shared {
+  uint64_t q_full, q_empty, mma_done;
+  uint64_t kv_full[8], kv_empty[8];
+  uint64_t s_full[NQT], p_full[NQT], o_full[NQT];
+  uint32_t tmem_base;
+  int abort;
+  int num_items;                     // items this CTA processes
+  int total_items;
+  int level_count[MAX_LEVELS];       // sequences with more than l 256-row blocks
+  int level_offset[MAX_LEVELS + 1];  // first item index of level (descending order)
+  int2 items[MAX_ITEMS_PER_CTA];     // (b, level << 16 | h)
+};
+
+template <int D>
+constexpr int smem_bytes() {
+  return Cfg<D>::SMEM_TILES + (int)sizeof(Shared) + 1024;
+}
+
+struct Params {
+  __nv_bfloat16* o;
+  float* lse;
+  const int32_t* cu_seqlens;
+  int B, Hq, Hkv, group, T;
+  int causal;
+  float scale_log2;  // softmax scale * log2(e)
+  int num_levels;    // ceil(max_seqlen / 256)
+};
+
+// Length of sequence b as the kernel uses it: an inconsistent cu_seqlens
+// entry reports a bounds error and makes the sequence empty.
+__device__ __forceinline__ void seq_range(const Params& p, int b, int& start, int& len) {
+  const int s = __ldg(p.cu_seqlens + b);
+  const int e = __ldg(p.cu_seqlens + b + 1);
+  if (s < 0 || e < s || e > p.T) {
+    start = 0;
+    len = 0;
+    return;
+  }
+  start = s;
+  len = e - s;
+}
+
+__device__ __forceinline__ int blocks_of(int len) { return (len + ROWS_PER_ITEM - 1) / ROWS_PER_ITEM; }
+
+// Work item w -> (b, level, h).  Items are ordered by descending level
+// (longest causal work first); within a level by sequence, then head.
+__device__ void decode_item(const Params& p, const Shared& sh, int w, int& b, int& level, int& h) {
+  // level_offset[k] is the first item of level num_levels-1-k; find the
+  // last k whose offset is <= w (empty levels share their successor's offset)
+  int a = 0, z = p.num_levels - 1;
+  while (a < z) {
+    const int mid = (a + z + 1) >> 1;
+    if (sh.level_offset[mid] <= w) a = mid; else z = mid - 1;
+  }
+  const int k = a;
+  level = p.num_levels - 1 - k;
+  const int r = w - sh.level_offset[k];
+  const int rank = r / p.Hq;
+  h = r - rank * p.Hq;
+  int seen = 0;
+  b = 0;
+  for (int i = 0; i < p.B; ++i) {
+    int st, len;
+    seq_range(p, i, st, len);
+    if (blocks_of(len) > level) {
+      if (seen == rank) {
+        b = i;
+        return;
+      }
+      ++seen;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* q_smem = smem + C::Q_OFF;
+  uint8_t* kv_smem = smem + C::KV_OFF;
+  Shared& sh = *reinterpret_cast<Shared*>(smem + C::SMEM_TILES);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int tid = threadIdx.x;
+
+  // ---------------- prologue: barriers, TMEM, work list ----------------
+  if (tid == 0) {
+    mbar_init(&sh.q_full, 1);
+    mbar_init(&sh.q_empty, 1);
+    mbar_init(&sh.mma_done, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&sh.kv_full[s], 1);
+      mbar_init(&sh.kv_empty[s], 1);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(&sh.s_full[t], 1);
+      mbar_init(&sh.p_full[t], BM);
+      mbar_init(&sh.o_full[t], 1);
+    }
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  for (int l = tid; l < p.num_levels; l += NUM_THREADS) sh.level_count[l] = 0;
+  __syncthreads();
+  for (int b = tid; b < p.B; b += NUM_THREADS) {
+    int st, len;
+    const int s = __ldg(p.cu_seqlens + b), e = __ldg(p.cu_seqlens + b + 1);
+    if (s < 0 || e < s || e > p.T || (b == 0 && s != 0)) report_error(kDevErrBounds);
+    seq_range(p, b, st, len);
+    int nb = blocks_of(len);
+    if (nb > p.num_levels) {
+      report_error(kDevErrBounds);
+      nb = p.num_levels;
+    }
+    // level l holds sequence b for every l < nb
+    for (int l = 0; l < nb; ++l) atomicAdd(&sh.level_count[l], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int k = 0; k < p.num_levels; ++k) {
+      sh.level_offset[k] = acc;
+      acc += sh.level_count[p.num_levels - 1 - k] * p.Hq;
+    }
+    sh.level_offset[p.num_levels] = acc;
+    sh.total_items = acc;
+    // zig-zag assignment: round r takes item r*G + (r even ? c : G-1-c)
+    const int G = gridDim.x, c = blockIdx.x;
+    int n = 0;
+    for (int r = 0;; ++r) {
+      const int w = r * G + ((r & 1) ? (G - 1 - c) : c);
+      if (w >= acc) break;
+      ++n;
+    }
+    if (n > MAX_ITEMS_PER_CTA) {
+      report_error(kDevErrBounds);
+      n = MAX_ITEMS_PER_CTA;
+    }
+    sh.num_items = n;
+  }
+  __syncthreads();
+  for (int i = tid; i < sh.num_items; i += NUM_THREADS) {
+    const int G = gridDim.x, c = blockIdx.x;
+    const int w = i * G + ((i & 1) ? (G - 1 - c) : c);
+    int b, level, h;
+    decode_item(p, sh, w, b, level, h);
+    sh.items[i] = make_int2(b, (level << 16) | h);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const int num_items = sh.num_items;
+  volatile int* abort = &sh.abort;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      uint32_t kv_it = 0, q_it = 0;
+      for (int it = 0; it < num_items && !*abort; ++it) {
+        const int2 item = sh.items[it];
+        const int b = item.x, level = item.y >> 16, h = item.y & 0xFFFF;
+        int start, len;
+        seq_range(p, b, start, len);
+        const int q0 = level * ROWS_PER_ITEM;
+        const int nkv_total = (len + BN - 1) / BN;
+        int nmax = 0;
+        for (int t = 0; t < NQT; ++t) {
+          const int rs = q0 + t * BM;
+          if (rs < len) nmax = p.causal ? min(nkv_total, rs / BN + 1) : nkv_total;
+        }
+        const int kh = h / p.group;
+        if (!mbar_wait(&sh.q_empty, (q_it & 1) ^ 1, abort)) break;
+        mbar_arrive_expect_tx(&sh.q_full, NQT * C::TILE_BYTES);
+        for (int t = 0; t < NQT; ++t)
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            tma_load_2d(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full,
+                        h * D + pn * 64, start + q0 + t * BM);
+        ++q_it;
+        for (int j = 0; j < nmax; ++j) {
+          for (int which = 0; which < 2; ++which) {
+            const uint32_t slot = kv_it % C::STAGES;
+            if (!mbar_wait(&sh.kv_empty[slot], ((kv_it / C::STAGES) & 1) ^ 1, abort)) break;
+            mbar_arrive_expect_tx(&sh.kv_full[slot], C::TILE_BYTES);
+            uint8_t* dst = kv_smem + slot * C::TILE_BYTES;
+            for (int pn = 0; pn < C::PANELS; ++pn)
+              tma_load_2d(dst + pn * C::PANEL_BYTES, which == 0 ? &tmK : &tmV, &sh.kv_full[slot],
+                          kh * D + pn * 64, start + j * BN);
+            ++kv_it;
+          }
+          if (*abort) break;
+        }
+      }
+      // Before the CTA can exit, every load issued must have landed (bounded
+      // wait that ignores the abort flag: the copies finish on their own).
+      for (uint32_t s = 0; s < (uint32_t)C::STAGES && s < kv_it; ++s) {
+        const uint32_t last = kv_it - 1 - ((kv_it - 1 - s) % C::STAGES);  // last use of slot
+        mbar_wait_bounded(&sh.kv_full[last % C::STAGES], (last / C::STAGES) & 1);
+      }
+      if (q_it > 0) mbar_wait_bounded(&sh.q_full, (q_it - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(q_smem);
+      const uint32_t kv_addr = smem_u32(kv_smem);
+      uint32_t kv_it = 0, q_it = 0;
+      uint32_t p_phase[NQT] = {0, 0};
+      bool ok = true;
+      for (int it = 0; it < num_items && ok; ++it) {
+        const int2 item = sh.items[it];
+        const int b = item.x, level = item.y >> 16;
+        int start, len;
+        seq_range(p, b, start, len);
+        (void)start;
+        const int q0 = level * ROWS_PER_ITEM;
+        const int nkv_total = (len + BN - 1) / BN;
+        int n[NQT];
+        int nmax = 0;
+        for (int t = 0; t < NQT; ++t) {
+          const int rs = q0 + t * BM;
+          n[t] = rs < len ? (p.causal ? min(nkv_total, rs / BN + 1) : nkv_total) : 0;
+          nmax = max(nmax, n[t]);
+        }
+        if (!mbar_wait(&sh.q_full, q_it & 1, abort)) { ok = false; break; }
+        ++q_it;
+        const uint32_t base = kv_it;
+        for (int j = 0; j <= nmax && ok; ++j) {
+          const uint32_t k_idx = base + 2 * j, v_idx = base + 2 * j - 1;
+          if (j < nmax &&
+              !mbar_wait(&sh.kv_full[k_idx % C::STAGES], (k_idx / C::STAGES) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          if (j >= 1 &&
+              !mbar_wait(&sh.kv_full[v_idx % C::STAGES], (v_idx / C::STAGES) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int t = 0; t < NQT; ++t) {
+            if (j >= 1 && j - 1 < n[t]) {
+              // O_t += P_t V_{j-1}   (A = P from TMEM, B = V, MN-major)
+              if (!mbar_wait(&sh.p_full[t], p_phase[t], abort)) { ok = false; break; }
+              p_phase[t] ^= 1;
+              tc_fence_after();
+              const uint32_t v_base = kv_addr + (v_idx % C::STAGES) * C::TILE_BYTES;
+              for (int kk = 0; kk < BN / 16; ++kk) {
+                const uint64_t bdesc = sdesc_sw128(v_base + kk * 16 * 128, C::PANEL_BYTES, 1024);
+                umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bdesc, C::IDESC_PV,
+                        (j - 1 > 0 || kk > 0) ? 1u : 0u);
+              }
+              if (j - 1 == n[t] - 1) umma_commit(&sh.o_full[t]);
+            }
+            if (j < n[t]) {
+              // S_t = Q_t K_j^T   (both K-major)
+              const uint32_t a_base = q_addr + t * C::TILE_BYTES;
+              const uint32_t b_base = kv_addr + (k_idx % C::STAGES) * C::TILE_BYTES;
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
+                umma_ss(tmem + t * 128, sdesc_sw128(a_base + off, 16, 1024),
+                        sdesc_sw128(b_base + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(&sh.s_full[t]);
+            }
+          }
+          if (!ok) break;
+          if (j >= 1) umma_commit(&sh.kv_empty[v_idx % C::STAGES]);
+          if (j < nmax) umma_commit(&sh.kv_empty[k_idx % C::STAGES]);
+        }
+        umma_commit(&sh.q_empty);
+        kv_it = base + 2 * nmax;
+      }
+      // every MMA issued must finish before TMEM is released
+      umma_commit(&sh.mma_done);
+      mbar_wait_bounded(&sh.mma_done, 0);
+    }
+  } else {
+    // ======================= softmax warpgroups =======================
+    const int t = (warp - 2) >> 2;          // query tile of this group
+    const int quarter = warp & 3;           // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;    // row of the tile owned by this thread
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_col = lane_base + t * 128;
+    const uint32_t o_col = lane_base + 256 + t * 128;
+    uint32_t s_phase = 0, o_phase = 0;
+    const float sl = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < num_items && ok; ++it) {
+      const int2 item = sh.items[it];
+      const int b = item.x, level = item.y >> 16, h = item.y & 0xFFFF;
+      int start, len;
+      seq_range(p, b, start, len);
+      const int rs = level * ROWS_PER_ITEM + t * BM;  // first row of this tile
+      if (rs >= len) continue;
+      const int nkv_total = (len + BN - 1) / BN;
+      const int n = p.causal ? min(nkv_total, rs / BN + 1) : nkv_total;
+      const int qpos = rs + row;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        if (!mbar_wait(&sh.s_full[t], s_phase, abort)) { ok = false; break; }
+        s_phase ^= 1;
+        tc_fence_after();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, s[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
+        const int kv0 = j * BN;
+        // masking: keys past the sequence end, and (causal) keys after the query
+        if (kv0 + BN > len || (p.causal && kv0 + BN - 1 > rs)) {
+          const int lim = min(len, p.causal ? qpos + 1 : len) - kv0;  // keys [0, lim) visible
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e >= lim) s[c][e] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
+        const float mx_s = mx * sl;
+        if (j == 0) {
+          m_ref = (mx_s == -INFINITY) ? 0.f : mx_s;
+        } else {
+          const bool need = mx_s > m_ref + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = fmaxf(m_ref, mx_s);
+            const float alpha = ex2(m_ref - m_new);
+            l *= alpha;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(o_col + c * 32, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(o_col + c * 32, o);
+            }
+            m_ref = m_new;
+          }
+        }
+        const float neg = -m_ref;
+        uint32_t pk[2][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(s[c][e]), sl, neg));
+            const float p1 = ex2(fmaf(__uint_as_float(s[c][e + 1]), sl, neg));
+            l += p0 + p1;
+            pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+          }
+        tmem_st32(s_col, pk[0]);
+        tmem_st32(s_col + 32, pk[1]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sh.p_full[t]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, LSE ----
+      if (!mbar_wait(&sh.o_full[t], o_phase, abort)) { ok = false; break; }
+      o_phase ^= 1;
+      tc_fence_after();
+      const bool valid = qpos < len;
+      const float inv_l = 1.f / l;
+      const size_t grow = (size_t)(start + qpos);
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (grow * p.Hq + h) * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_col + c * 32, o);
+        tmem_ld_wait(o);
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[c * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        }
+      }
+      if (valid && p.lse) p.lse[(size_t)h * p.T + grow] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+      tc_fence_before();
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace prefill
+}  // namespace fa

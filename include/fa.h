@@ -1,0 +1,154 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact IO-aware attention forward on B200 (sm_100a).
+ *
+ * The operation (definition, "FlashAttention-3 vs naive attention", cnblogs,
+ * section 1.1; "FlashAttention" concept page, Definition):
+ *
+ *     O = softmax(Q K^T * scale + mask) V
+ *
+ * computed tile by tile with an online softmax (running row max m and sum l,
+ * "gsyq.cn FA vs FIA" section 1), so the L x L score matrix never reaches
+ * device memory.  Two modes:
+ *   - fa_prefill: packed variable-length sequences ("flash-attention" skill
+ *     page, section 3.4), optional causal mask (section 3.2), grouped kv heads
+ *     (GQA/MQA appendix).
+ *   - fa_decode_paged: one query token per request against a paged KV cache
+ *     addressed by a block table (PagedAttention appendix), split along the
+ *     context and merged by log-sum-exp (FlashDecoding / Split-KV appendix).
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *     keeps no pointer after returning.  Tensors are dense, row-major in the
+ *     layout stated beside each argument, 16-byte aligned.
+ *   - bf16 means IEEE bfloat16 (2 bytes); fp32 means IEEE binary32.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream); no call synchronises the host except fa_get_device_error.
+ *   - Argument checks happen on the host before any launch; a failed check
+ *     returns FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED and launches nothing.
+ *   - Values that only the device can see (cu_seqlens, seq_lens, block_table
+ *     entries) are range-checked in the kernels: an out-of-range value never
+ *     causes an out-of-bounds access; it sets a sticky device error word
+ *     (FA_ERR_DEVICE_BOUNDS) and the affected rows are skipped or read as
+ *     zero.  Every wait inside a kernel is bounded in time; on timeout the
+ *     kernel sets FA_ERR_DEVICE_TIMEOUT and returns.  Read the word with
+ *     fa_get_device_error.
+ *   - head_dim d must be 64 or 128 on the bf16 paths; Hq % Hkv == 0.
+ *   - scale <= 0 selects the default 1/sqrt(d) (skill page, section 3.2,
+ *     softmax_scale=None).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,    /* null pointer, bad shape, misalignment       */
+    FA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. d = 96)     */
+    FA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed        */
+    FA_ERR_DEVICE_BOUNDS = 4,  /* a kernel saw an out-of-range index          */
+    FA_ERR_DEVICE_TIMEOUT = 5  /* a kernel wait ran past its time limit       */
+} fa_status;
+
+/*
+ * Prefill: exact attention over B packed sequences.
+ *
+ *   q           bf16 [T, Hq, d]   query rows; token t of sequence b is row
+ *                                 cu_seqlens[b] + i, i in [0, L_b)
+ *   k, v        bf16 [T, Hkv, d]  key / value rows, same packing
+ *   o           bf16 [T, Hq, d]   output (written)
+ *   lse         fp32 [Hq, T]      natural-log log-sum-exp of each row's scaled
+ *                                 scores (written), or NULL
+ *   cu_seqlens  int32 [B+1]       device; cu_seqlens[0] = 0, nondecreasing,
+ *                                 cu_seqlens[B] = T
+ *   causal      nonzero: query i sees keys j <= i of its own sequence;
+ *               zero: it sees all L_b keys of its own sequence
+ *   scale       multiplier of Q K^T (<= 0: 1/sqrt(d))
+ *   total_tokens  T (host copy of cu_seqlens[B]; sizes q/k/v/o)
+ *   max_seqlen    an upper bound on every L_b (host; sizes the grid)
+ * Query head h reads kv head h / (Hq / Hkv).  A sequence with L_b = 0 is
+ * skipped.  Does not allocate.
+ */
+fa_status fa_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                     const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                     float scale, fa_stream_t stream, int total_tokens, int max_seqlen);
+
+/*
+ * Paged decode: one query token per request at the end of its context.
+ *
+ *   q            bf16 [B, Hq, d]
+ *   k_pages,
+ *   v_pages      bf16 [num_pages, page_size, Hkv, d]   the page pool
+ *   block_table  int32 [B, max_blocks_per_seq]  device; entry i of row b is
+ *                the pool page holding tokens [i*page_size, (i+1)*page_size)
+ *                of request b.  Entries at i >= ceil(seq_lens[b]/page_size)
+ *                are never read.
+ *   seq_lens     int32 [B]  device; context length of each request,
+ *                0 <= seq_lens[b] <= max_blocks_per_seq * page_size
+ *   page_size    tokens per page (>= 1)
+ *   num_splits   number of contiguous page ranges each request's context is
+ *                cut into (0 = choose automatically, see
+ *                fa_decode_auto_splits); the result does not depend on it
+ *                beyond rounding
+ *   o            bf16 [B, Hq, d]  output (written)
+ *   lse          fp32 [B, Hq]  natural-log log-sum-exp, or NULL
+ *   workspace    device scratch of at least
+ *                fa_decode_workspace_size(B, Hq, d, resolved num_splits)
+ *                bytes, 256-byte aligned; NULL = the library allocates it
+ *                stream-ordered (cudaMallocAsync/cudaFreeAsync on `stream`)
+ * A request with seq_lens[b] = 0 yields O = 0 and LSE = -inf.  Requires
+ * Hq / Hkv <= 8.
+ */
+fa_status fa_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                          const int32_t *block_table, const int32_t *seq_lens, int page_size,
+                          int num_splits, void *o, fa_stream_t stream, int B, int Hq, int Hkv,
+                          int d, int max_blocks_per_seq, int num_pages, float scale, float *lse,
+                          void *workspace, size_t workspace_bytes);
+
+/* Bytes of workspace fa_decode_paged needs for this shape and split count
+ * (partial outputs fp32 [B, Hq, S, d] and partial LSEs fp32 [B, Hq, S]). */
+size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits);
+
+/* The split count num_splits = 0 resolves to: enough (request, split) work
+ * units to give every SM several to run, and no more splits than the
+ * longest context has pages.  num_sms <= 0 queries the current device. */
+int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int num_sms);
+
+/*
+ * fp32 debug paths: the same operations with fp32 q/k/v/o (layouts as
+ * above), plain CUDA-core arithmetic, any d in [1, 256].  For checking
+ * conventions at fp32 precision, not for speed.
+ */
+fa_status fa_prefill_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+                         const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                         float scale, fa_stream_t stream, int total_tokens, int max_seqlen);
+
+fa_status fa_decode_paged_f32(const float *q, const float *k_pages, const float *v_pages,
+                              const int32_t *block_table, const int32_t *seq_lens,
+                              int page_size, float *o, fa_stream_t stream, int B, int Hq,
+                              int Hkv, int d, int max_blocks_per_seq, int num_pages,
+                              float scale, float *lse);
+
+/* Reads and clears the sticky device error word of the current device
+ * (synchronises `stream` first).  *code receives FA_OK or the first
+ * FA_ERR_DEVICE_* recorded.  Returns FA_ERR_CUDA if the read fails. */
+fa_status fa_get_device_error(fa_stream_t stream, int *code);
+
+/* Static description of a status code. */
+const char *fa_get_error_string(fa_status status);
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,33 @@
+"""Comparison helpers for the GPU-versus-oracle parity tests.
+
+Tolerances: bf16 outputs within max-abs 1e-2 and mean-abs 1e-3 of the fp64
+oracle, LSE within 1e-3; the fp32 debug path within 1e-5.
+"""
+import numpy as np
+
+BF16_MAX_ABS = 1e-2
+BF16_MEAN_ABS = 1e-3
+LSE_ABS = 1e-3
+F32_ABS = 1e-5
+
+
+def to_np(t):
+    return t.detach().float().cpu().double().numpy() if hasattr(t, "detach") else np.asarray(t)
+
+
+def check_close(got, ref, max_abs, mean_abs=None, what="output"):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, f"{what}: shape {got.shape} vs {ref.shape}"
+    assert np.isfinite(got).all() == np.isfinite(ref).all() or (
+        np.array_equal(np.isfinite(got), np.isfinite(ref))), f"{what}: non-finite mismatch"
+    fin = np.isfinite(ref)
+    # -inf must match -inf exactly (empty rows)
+    assert np.array_equal(got[~fin], ref[~fin]), f"{what}: non-finite entries differ"
+    if fin.any():
+        err = np.abs(got[fin] - ref[fin])
+        assert err.max() <= max_abs, f"{what}: max abs err {err.max():.3e} > {max_abs:.1e}"
+        if mean_abs is not None:
+            assert err.mean() <= mean_abs, f"{what}: mean abs err {err.mean():.3e} > {mean_abs:.1e}"
+        return float(err.max()), float(err.mean())
+    return 0.0, 0.0

@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI: the library builds for sm_100a, loads
+without a GPU, exports every symbol ``include/fa.h`` declares, and rejects
+bad arguments before touching the device.  No call here reaches a kernel
+launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_86_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails validation first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.ensure_built()
+    return api.load_library()
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("fa_prefill", "fa_decode_paged", "fa_decode_workspace_size",
+              "fa_decode_auto_splits", "fa_get_error_string", "fa_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_library_is_built_for_sm100a():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
+
+
+def test_error_strings(lib):
+    for code in range(6):
+        assert api.error_string(code)
+    assert api.error_string(99) == "unknown status"
+
+
+def _prefill(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, cu=FAKE, B=1, Hq=4, Hkv=2, d=128,
+             causal=1, scale=0.0, stream=None, T=16, maxlen=16)
+    a.update(kw)
+    return lib.fa_prefill(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu"], a["B"], a["Hq"],
+                          a["Hkv"], a["d"], a["causal"], a["scale"], a["stream"], a["T"],
+                          a["maxlen"])
+
+
+def test_prefill_argument_checks(lib):
+    assert _prefill(lib, q=None) == api.FA_ERR_INVALID_ARG
+    assert _prefill(lib, cu=None) == api.FA_ERR_INVALID_ARG
+    assert _prefill(lib, Hq=6, Hkv=4) == api.FA_ERR_INVALID_ARG      # Hq % Hkv
+    assert _prefill(lib, B=-1) == api.FA_ERR_INVALID_ARG
+    assert _prefill(lib, T=-5) == api.FA_ERR_INVALID_ARG
+    assert _prefill(lib, q=ctypes.c_void_p(0x1008)) == api.FA_ERR_INVALID_ARG  # misaligned
+    assert _prefill(lib, d=96) == api.FA_ERR_UNSUPPORTED
+    assert _prefill(lib, d=256) == api.FA_ERR_UNSUPPORTED
+    assert _prefill(lib, maxlen=1024 * 256 + 1) == api.FA_ERR_UNSUPPORTED
+    # empty problems are a no-op (no launch)
+    assert _prefill(lib, B=0) == api.FA_OK
+    assert _prefill(lib, T=0) == api.FA_OK
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, ps=16, S=0, o=FAKE, stream=None, B=2,
+             Hq=32, Hkv=8, d=128, maxb=4, npages=8, scale=0.0, lse=None, ws=None, wsb=0)
+    a.update(kw)
+    return lib.fa_decode_paged(a["q"], a["k"], a["v"], a["bt"], a["sl"], a["ps"], a["S"], a["o"],
+                               a["stream"], a["B"], a["Hq"], a["Hkv"], a["d"], a["maxb"],
+                               a["npages"], a["scale"], a["lse"], a["ws"], a["wsb"])
+
+
+def test_decode_argument_checks(lib):
+    assert _decode(lib, bt=None) == api.FA_ERR_INVALID_ARG
+    assert _decode(lib, ps=0) == api.FA_ERR_INVALID_ARG
+    assert _decode(lib, S=-1) == api.FA_ERR_INVALID_ARG
+    assert _decode(lib, Hq=12, Hkv=8) == api.FA_ERR_INVALID_ARG
+    assert _decode(lib, ws=ctypes.c_void_p(0x1010)) == api.FA_ERR_INVALID_ARG  # not 256-aligned
+    assert _decode(lib, d=80) == api.FA_ERR_UNSUPPORTED
+    assert _decode(lib, Hq=32, Hkv=2) == api.FA_ERR_UNSUPPORTED          # group 16 > 8
+    assert _decode(lib, ps=8) == api.FA_ERR_UNSUPPORTED                  # not a multiple of 16
+    # explicit workspace that is too small
+    need = lib.fa_decode_workspace_size(2, 32, 128, 4)
+    assert _decode(lib, S=4, ws=ctypes.c_void_p(0x10000), wsb=need - 1) == api.FA_ERR_INVALID_ARG
+    assert _decode(lib, B=0) == api.FA_OK
+
+
+def test_decode_workspace_is_linear_in_splits_not_context(lib):
+    """The split workspace holds fp32 partial outputs and LSEs:
+    B*Hq*S*(d+1) floats (rounded to 256-byte blocks), independent of the
+    context length -- nothing of size N^2 (or even N) is ever allocated."""
+    for B, Hq, d, S in ((64, 32, 128, 10), (2, 32, 128, 296), (1, 1, 64, 2)):
+        n = lib.fa_decode_workspace_size(B, Hq, d, S)
+        assert n >= B * Hq * S * (d + 1) * 4
+        assert n <= B * Hq * S * (d + 1) * 4 + 512
+    assert lib.fa_decode_workspace_size(64, 32, 128, 1) == 0
+
+
+def test_auto_splits_rule(lib):
+    # enough (request, split) units for several per SM, capped by the page count
+    assert lib.fa_decode_auto_splits(64, 8, 2048, 148) == 10
+    assert lib.fa_decode_auto_splits(2, 8, 2048, 148) == 296
+    assert lib.fa_decode_auto_splits(2, 8, 3, 148) == 3
+    assert lib.fa_decode_auto_splits(10000, 8, 64, 148) == 1
+
+
+def test_python_binding_rejects_host_tensors():
+    import torch
+    q = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        api.fa_prefill(q, q[:, :1], q[:, :1], q, None, cu, True)
