@@ -170,7 +170,9 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
     float acc[C::KS][4];
 #pragma unroll
     for (int mt = 0; mt < C::KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // query heads 2tq, 2tq+1
+    // query heads 2tq, 2tq+1: running max, exact sum of exp (for the LSE) and
+    // sum of the bf16-rounded weights the PV MMA uses (normalises O)
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
     const float sl = p.scale_log2;
     const uint32_t sbase = smem_u32(smem);
 
@@ -219,8 +221,12 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
       const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);    // ex2(-inf) = 0
       const float p00 = ex2(s00 - mn0), p01 = ex2(s01 - mn1);
       const float p10 = ex2(s10 - mn0), p11 = ex2(s11 - mn1);
-      l0 = l0 * al0 + p00 + p10;
-      l1 = l1 * al1 + p01 + p11;
+      // P^T in bf16 (the MMA operand); the row sums use the same rounded values
+      const uint32_t x0 = pack_bf16x2(p00, p01), x1 = pack_bf16x2(p10, p11);
+      l0 = l0 * al0 + (p00 + p10);
+      l1 = l1 * al1 + (p01 + p11);
+      r0 = r0 * al0 + (__uint_as_float(x0 << 16) + __uint_as_float(x1 << 16));
+      r1 = r1 * al1 + (__uint_as_float(x0 & 0xFFFF0000u) + __uint_as_float(x1 & 0xFFFF0000u));
       m0 = mn0;
       m1 = mn1;
 #pragma unroll
@@ -231,8 +237,8 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
         acc[mt][3] *= al1;
       }
       // P^T as the MMA B operand (k = token, n = query head)
-      const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p00, p01));
-      const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p10, p11));
+      const uint32_t pb0 = movmatrix_trans(x0);
+      const uint32_t pb1 = movmatrix_trans(x1);
       // ---- O^T[d][n] += sum_tok V[tok][d] P[n][tok] ----
 #pragma unroll
       for (int mt = 0; mt < C::KS; ++mt) {
@@ -252,8 +258,10 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
     for (int off = 4; off < 32; off <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, off);
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      r0 += __shfl_xor_sync(0xffffffffu, r0, off);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, off);
     }
-    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    const float inv0 = r0 > 0.f ? 1.f / r0 : 0.f, inv1 = r1 > 0.f ? 1.f / r1 : 0.f;
     const float ln2 = 0.69314718055994531f;
     const float lse0 = l0 > 0.f ? (m0 + __log2f(l0)) * ln2 : -INFINITY;
     const float lse1 = l1 > 0.f ? (m1 + __log2f(l1)) * ln2 : -INFINITY;

@@ -127,6 +127,14 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   const int smem = smem_bytes<D>();
   static bool attr_ok = set_smem(prefill_kernel<D>, smem);
   if (!attr_ok) return FA_ERR_CUDA;
+  // The kernel hands registers between its warpgroups with setmaxnreg; the
+  // split only fits if the launch allots kRegsLaunch registers per thread
+  // (otherwise setmaxnreg.inc could never be satisfied).
+  static int launch_regs = [] {
+    cudaFuncAttributes a;
+    return cudaFuncGetAttributes(&a, prefill_kernel<D>) == cudaSuccess ? a.numRegs : -1;
+  }();
+  if (launch_regs < (int)kRegsLaunch) return FA_ERR_UNSUPPORTED;
   prefill_kernel<D><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -12,12 +12,14 @@
 //   memory as bf16, and the tensor cores accumulate O += P V_j in tensor
 //   memory.  At the end O / l is stored as bf16 and LSE = ln2*(m + log2 l).
 //
-// CTA layout (320 threads, one CTA per SM, persistent):
+// CTA layout (384 threads = 3 warpgroups, one CTA per SM, persistent):
 //   warp 0      TMA producer: Q tiles once per work item, then K_j, V_j
 //               alternately through a ring of 128 x D smem slots
 //   warp 1      MMA issuer (one thread) and TMEM owner (512 columns)
-//   warps 2-5   softmax for query tile 0 (rows q0 .. q0+127)
-//   warps 6-9   softmax for query tile 1 (rows q0+128 .. q0+255)
+//   warps 2-3   idle (they complete the first warpgroup)
+//   warps 4-7   softmax for query tile 0 (rows q0 .. q0+127)
+//   warps 8-11  softmax for query tile 1 (rows q0+128 .. q0+255)
+// setmaxnreg moves registers from the first warpgroup to the softmax ones.
 // The two query tiles share every K/V tile, and while one softmax group
 // works on its S the tensor cores run the other tile's P V and Q K^T.
 //
@@ -30,6 +32,13 @@
 // exceeds it by more than 8 (log2 units), so P <= 256 and O is rescaled in
 // tensor memory only on those (rare) tiles.  The final O / l and the LSE use
 // the same reference max, so the result is exact up to rounding.
+//
+// Softmax arithmetic per score: one three-input max per two scores, one
+// packed FMA per two scores for s*scale*log2e - m, 2^x on the MUFU unit for
+// three of every four pairs and on the FMA pipe (exp2_fma_pair) for the
+// fourth, which balances the two units.  P is rounded to bf16 for the MMA;
+// O is divided by the sum of those rounded values (so O is a weighted mean
+// with exactly the weights used) and the LSE uses the unrounded sum.
 #pragma once
 
 #include "ptx.cuh"
@@ -41,8 +50,16 @@ constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 128;           // keys per K/V tile
 constexpr int NQT = 2;            // query tiles per work item
 constexpr int ROWS_PER_ITEM = NQT * BM;
-constexpr int NUM_WARPS = 10;
+constexpr int NUM_WARPS = 12;  // 3 warpgroups: control (producer, MMA, 2 idle), softmax x2
 constexpr int NUM_THREADS = NUM_WARPS * 32;
+// Register split between the warpgroups (setmaxnreg).  The launch allots
+// kRegsLaunch per thread; the control group gives most of its share to the
+// softmax groups: 128*kRegsControl + 256*kRegsSoftmax <= 384*kRegsLaunch.
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsControl = 64;
+constexpr uint32_t kRegsSoftmax = 216;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= NUM_THREADS * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int MAX_LEVELS = 1024;  // max_seqlen <= 1024 * 256
@@ -231,7 +248,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int num_items = sh.num_items;
   volatile int* abort = &sh.abort;
 
-  if (warp == 0) {
+  if (warp < 4) {
+    // ---- warpgroup 0: producer (warp 0), MMA issuer (warp 1), warps 2-3 idle ----
+    setmaxnreg_dec<kRegsControl>();
+   if (warp == 0) {
     // ======================= TMA producer =======================
     if (lane == 0) {
       uint32_t kv_it = 0, q_it = 0;
@@ -243,31 +263,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int q0 = level * ROWS_PER_ITEM;
         const int nkv_total = (len + BN - 1) / BN;
         int nmax = 0;
+#pragma unroll
         for (int t = 0; t < NQT; ++t) {
           const int rs = q0 + t * BM;
           if (rs < len) nmax = p.causal ? min(nkv_total, rs / BN + 1) : nkv_total;
         }
         const int kh = h / p.group;
+        // K/V tile loads of this item; the first pair goes out before the
+        // wait for the Q buffer, so it overlaps the previous item's tail
+        int next = 0;  // next K/V load (2*j + which) to issue
+        auto issue_kv = [&](int upto) -> bool {
+          for (; next < upto; ++next) {
+            const uint32_t slot = kv_it % C::STAGES;
+            if (!mbar_wait(&sh.kv_empty[slot], ((kv_it / C::STAGES) & 1) ^ 1, abort)) return false;
+            mbar_arrive_expect_tx(&sh.kv_full[slot], C::TILE_BYTES);
+            uint8_t* dst = kv_smem + slot * C::TILE_BYTES;
+            const CUtensorMap* m = (next & 1) ? &tmV : &tmK;
+#pragma unroll
+            for (int pn = 0; pn < C::PANELS; ++pn)
+              tma_load_2d(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot], kh * D + pn * 64,
+                          start + (next >> 1) * BN);
+            ++kv_it;
+          }
+          return true;
+        };
+        if (!issue_kv(min(2, 2 * nmax))) break;
         if (!mbar_wait(&sh.q_empty, (q_it & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&sh.q_full, NQT * C::TILE_BYTES);
+#pragma unroll
         for (int t = 0; t < NQT; ++t)
+#pragma unroll
           for (int pn = 0; pn < C::PANELS; ++pn)
             tma_load_2d(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full,
                         h * D + pn * 64, start + q0 + t * BM);
         ++q_it;
-        for (int j = 0; j < nmax; ++j) {
-          for (int which = 0; which < 2; ++which) {
-            const uint32_t slot = kv_it % C::STAGES;
-            if (!mbar_wait(&sh.kv_empty[slot], ((kv_it / C::STAGES) & 1) ^ 1, abort)) break;
-            mbar_arrive_expect_tx(&sh.kv_full[slot], C::TILE_BYTES);
-            uint8_t* dst = kv_smem + slot * C::TILE_BYTES;
-            for (int pn = 0; pn < C::PANELS; ++pn)
-              tma_load_2d(dst + pn * C::PANEL_BYTES, which == 0 ? &tmK : &tmV, &sh.kv_full[slot],
-                          kh * D + pn * 64, start + j * BN);
-            ++kv_it;
-          }
-          if (*abort) break;
-        }
+        if (!issue_kv(2 * nmax)) break;
       }
       // Before the CTA can exit, every load issued must have landed (bounded
       // wait that ignores the abort flag: the copies finish on their own).
@@ -277,14 +307,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (q_it > 0) mbar_wait_bounded(&sh.q_full, (q_it - 1) & 1);
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(q_smem);
       const uint32_t kv_addr = smem_u32(kv_smem);
       uint32_t kv_it = 0, q_it = 0;
-      uint32_t p_phase[NQT] = {0, 0};
+      uint32_t p_phase0 = 0, p_phase1 = 0;
       bool ok = true;
+      // O_t += P_t V   (A = P from TMEM, B = V, MN-major)
+      auto issue_pv = [&](int t, uint32_t v_idx, bool first) {
+        const uint32_t v_base = kv_addr + (v_idx % C::STAGES) * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bdesc = sdesc_sw128(v_base + kk * 16 * 128, C::PANEL_BYTES, 1024);
+          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bdesc, C::IDESC_PV,
+                  (!first || kk > 0) ? 1u : 0u);
+        }
+      };
+      // S_t = Q_t K^T   (both K-major)
+      auto issue_s = [&](int t, uint32_t k_idx) {
+        const uint32_t a_base = q_addr + t * C::TILE_BYTES;
+        const uint32_t b_base = kv_addr + (k_idx % C::STAGES) * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + t * 128, sdesc_sw128(a_base + off, 16, 1024),
+                  sdesc_sw128(b_base + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
       for (int it = 0; it < num_items && ok; ++it) {
         const int2 item = sh.items[it];
         const int b = item.x, level = item.y >> 16;
@@ -293,17 +344,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         (void)start;
         const int q0 = level * ROWS_PER_ITEM;
         const int nkv_total = (len + BN - 1) / BN;
-        int n[NQT];
-        int nmax = 0;
-        for (int t = 0; t < NQT; ++t) {
-          const int rs = q0 + t * BM;
-          n[t] = rs < len ? (p.causal ? min(nkv_total, rs / BN + 1) : nkv_total) : 0;
-          nmax = max(nmax, n[t]);
-        }
+        const int n0 = q0 < len ? (p.causal ? min(nkv_total, q0 / BN + 1) : nkv_total) : 0;
+        const int n1 = q0 + BM < len ? (p.causal ? min(nkv_total, (q0 + BM) / BN + 1) : nkv_total) : 0;
+        const int nmax = max(n0, n1);
         if (!mbar_wait(&sh.q_full, q_it & 1, abort)) { ok = false; break; }
         ++q_it;
         const uint32_t base = kv_it;
-        for (int j = 0; j <= nmax && ok; ++j) {
+        for (int j = 0; j <= nmax; ++j) {
           const uint32_t k_idx = base + 2 * j, v_idx = base + 2 * j - 1;
           if (j < nmax &&
               !mbar_wait(&sh.kv_full[k_idx % C::STAGES], (k_idx / C::STAGES) & 1, abort)) {
@@ -316,46 +363,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          for (int t = 0; t < NQT; ++t) {
-            if (j >= 1 && j - 1 < n[t]) {
-              // O_t += P_t V_{j-1}   (A = P from TMEM, B = V, MN-major)
-              if (!mbar_wait(&sh.p_full[t], p_phase[t], abort)) { ok = false; break; }
-              p_phase[t] ^= 1;
-              tc_fence_after();
-              const uint32_t v_base = kv_addr + (v_idx % C::STAGES) * C::TILE_BYTES;
-              for (int kk = 0; kk < BN / 16; ++kk) {
-                const uint64_t bdesc = sdesc_sw128(v_base + kk * 16 * 128, C::PANEL_BYTES, 1024);
-                umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bdesc, C::IDESC_PV,
-                        (j - 1 > 0 || kk > 0) ? 1u : 0u);
-              }
-              if (j - 1 == n[t] - 1) umma_commit(&sh.o_full[t]);
-            }
-            if (j < n[t]) {
-              // S_t = Q_t K_j^T   (both K-major)
-              const uint32_t a_base = q_addr + t * C::TILE_BYTES;
-              const uint32_t b_base = kv_addr + (k_idx % C::STAGES) * C::TILE_BYTES;
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-                umma_ss(tmem + t * 128, sdesc_sw128(a_base + off, 16, 1024),
-                        sdesc_sw128(b_base + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
-              }
-              umma_commit(&sh.s_full[t]);
-            }
+          // tile 0
+          if (j >= 1 && j - 1 < n0) {
+            if (!mbar_wait(&sh.p_full[0], p_phase0, abort)) { ok = false; break; }
+            p_phase0 ^= 1;
+            tc_fence_after();
+            issue_pv(0, v_idx, j == 1);
+            if (j == n0) umma_commit(&sh.o_full[0]);
           }
-          if (!ok) break;
+          if (j < n0) {
+            issue_s(0, k_idx);
+            umma_commit(&sh.s_full[0]);
+          }
+          // tile 1
+          if (j >= 1 && j - 1 < n1) {
+            if (!mbar_wait(&sh.p_full[1], p_phase1, abort)) { ok = false; break; }
+            p_phase1 ^= 1;
+            tc_fence_after();
+            issue_pv(1, v_idx, j == 1);
+            if (j == n1) umma_commit(&sh.o_full[1]);
+          }
+          if (j < n1) {
+            issue_s(1, k_idx);
+            umma_commit(&sh.s_full[1]);
+          }
           if (j >= 1) umma_commit(&sh.kv_empty[v_idx % C::STAGES]);
           if (j < nmax) umma_commit(&sh.kv_empty[k_idx % C::STAGES]);
+          if (j == nmax - 1 || nmax == 0) umma_commit(&sh.q_empty);  // last S of the item issued
         }
-        umma_commit(&sh.q_empty);
         kv_it = base + 2 * nmax;
       }
       // every MMA issued must finish before TMEM is released
       umma_commit(&sh.mma_done);
       mbar_wait_bounded(&sh.mma_done, 0);
     }
+   }
   } else {
     // ======================= softmax warpgroups =======================
-    const int t = (warp - 2) >> 2;          // query tile of this group
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int t = (warp - 4) >> 2;          // query tile of this group
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // row of the tile owned by this thread
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -363,6 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t o_col = lane_base + 256 + t * 128;
     uint32_t s_phase = 0, o_phase = 0;
     const float sl = p.scale_log2;
+    const uint64_t sl2 = f2_pack(sl, sl);
     bool ok = true;
     for (int it = 0; it < num_items && ok; ++it) {
       const int2 item = sh.items[it];
@@ -374,7 +421,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int nkv_total = (len + BN - 1) / BN;
       const int n = p.causal ? min(nkv_total, rs / BN + 1) : nkv_total;
       const int qpos = rs + row;
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY;
+      // row sums, each as two interleaved fp32 pairs: le = exact sum of
+      // exp (for the LSE), lr = sum of the bf16 values the PV MMA consumes
+      // (normalises O consistently with its own weights)
+      uint64_t le_a = 0, le_b = 0, lr_a = 0, lr_b = 0;
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait(&sh.s_full[t], s_phase, abort)) { ok = false; break; }
         s_phase ^= 1;
@@ -392,47 +443,86 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (c * 32 + e >= lim) s[c][e] = __float_as_uint(-INFINITY);
+              s[c][e] = (c * 32 + e >= lim) ? __float_as_uint(-INFINITY) : s[c][e];
         }
-        float mx = -INFINITY;
+        // row max: four independent chains of three-input maxima
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
-        const float mx_s = mx * sl;
+          for (int e = 0; e < 32; e += 8) {
+            mx0 = fmax3(mx0, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+            mx1 = fmax3(mx1, __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
+            mx2 = fmax3(mx2, __uint_as_float(s[c][e + 4]), __uint_as_float(s[c][e + 5]));
+            mx3 = fmax3(mx3, __uint_as_float(s[c][e + 6]), __uint_as_float(s[c][e + 7]));
+          }
+        const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
+        float alpha = 1.f;
+        bool rescale = false;
         if (j == 0) {
           m_ref = (mx_s == -INFINITY) ? 0.f : mx_s;
-        } else {
-          const bool need = mx_s > m_ref + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, need)) {
-            const float m_new = fmaxf(m_ref, mx_s);
-            const float alpha = ex2(m_ref - m_new);
-            l *= alpha;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(o_col + c * 32, o);
-              tmem_ld_wait(o);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(o_col + c * 32, o);
-            }
-            m_ref = m_new;
-          }
+        } else if (__any_sync(0xffffffffu, mx_s > m_ref + kRescaleThreshold)) {
+          const float m_new = fmaxf(m_ref, mx_s);
+          alpha = ex2(m_ref - m_new);
+          const uint64_t a2 = f2_pack(alpha, alpha);
+          le_a = f2_mul(le_a, a2);
+          le_b = f2_mul(le_b, a2);
+          lr_a = f2_mul(lr_a, a2);
+          lr_b = f2_mul(lr_b, a2);
+          m_ref = m_new;
+          rescale = true;
         }
-        const float neg = -m_ref;
-        uint32_t pk[2][32];
+        // P = 2^(s*scale*log2e - m): three of every four pairs on MUFU, one on
+        // the FMA pipe; packed bf16 pairs overwrite s[c][0..15] in order
+        const uint64_t neg2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[c][e]), sl, neg));
-            const float p1 = ex2(fmaf(__uint_as_float(s[c][e + 1]), sl, neg));
-            l += p0 + p1;
-            pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+            const uint64_t x =
+                f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), sl2, neg2);
+            uint64_t pr;
+            if (((e >> 1) & 3) == 3) {
+              pr = exp2_fma_pair(x);
+            } else {
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              pr = f2_pack(ex2(x0), ex2(x1));
+            }
+            float p0, p1;
+            f2_unpack(pr, p0, p1);
+            const uint32_t pp = pack_bf16x2(p0, p1);
+            const uint64_t pq =
+                f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xFFFF0000u));
+            if ((e >> 1) & 1) {
+              le_b = f2_add(le_b, pr);
+              lr_b = f2_add(lr_b, pq);
+            } else {
+              le_a = f2_add(le_a, pr);
+              lr_a = f2_add(lr_a, pq);
+            }
+            s[c][e >> 1] = pp;
           }
-        tmem_st32(s_col, pk[0]);
-        tmem_st32(s_col + 32, pk[1]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(s_col + c * 16, s[c]);
+        if (rescale) {
+          // O *= alpha; PV_t(j-1) has completed (it precedes S_t(j) in issue order)
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_col + c * 32, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float o0, o1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
+              o[e] = __float_as_uint(o0);
+              o[e + 1] = __float_as_uint(o1);
+            }
+            tmem_st32(o_col + c * 32, o);
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sh.p_full[t]);
@@ -442,8 +532,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&sh.o_full[t], o_phase, abort)) { ok = false; break; }
       o_phase ^= 1;
       tc_fence_after();
+      float la0, la1, lb0, lb1;
+      f2_unpack(le_a, la0, la1);
+      f2_unpack(le_b, lb0, lb1);
+      const float l_exact = (la0 + la1) + (lb0 + lb1);
+      f2_unpack(lr_a, la0, la1);
+      f2_unpack(lr_b, lb0, lb1);
+      const float l_round = (la0 + la1) + (lb0 + lb1);
       const bool valid = qpos < len;
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / l_round;
       const size_t grow = (size_t)(start + qpos);
       uint4* dst = reinterpret_cast<uint4*>(p.o + (grow * p.Hq + h) * D);
 #pragma unroll
@@ -461,7 +558,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             dst[c * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
         }
       }
-      if (valid && p.lse) p.lse[(size_t)h * p.T + grow] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+      if (valid && p.lse)
+        p.lse[(size_t)h * p.T + grow] = (m_ref + __log2f(l_exact)) * 0.69314718055994531f;
       tc_fence_before();
     }
   }

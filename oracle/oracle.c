@@ -196,9 +196,9 @@ int oracle_prefill(const void *q, const void *k, const void *v, int dtype,
         return -1;
     int64_t T = cu_seqlens[B];
     int64_t nrows = T * Hq;
-    int64_t *rt = (int64_t *)malloc((size_t)(nrows > 0 ? nrows : 1) * sizeof(int64_t));
-    int32_t *rh = (int32_t *)malloc((size_t)(nrows > 0 ? nrows : 1) * sizeof(int32_t));
-    double *l = (double *)malloc((size_t)(nrows > 0 ? nrows : 1) * sizeof(double));
+    int64_t *rt = (int64_t *)calloc((size_t)(nrows > 0 ? nrows : 1), sizeof(int64_t));
+    int32_t *rh = (int32_t *)calloc((size_t)(nrows > 0 ? nrows : 1), sizeof(int32_t));
+    double *l = (double *)calloc((size_t)(nrows > 0 ? nrows : 1), sizeof(double));
     if (!rt || !rh || !l) {
         free(rt);
         free(rh);

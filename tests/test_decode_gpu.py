@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from exact_io_aware_86_b200 import api, inputs
-from parity import BF16_MAX_ABS, BF16_MEAN_ABS, F32_ABS, LSE_ABS, check_close, to_np
+from parity import BF16_MAX_ABS, BF16_MEAN_ABS, F32_ABS, LSE_ABS, check_bf16, check_close, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +32,7 @@ def reference(inp):
 def assert_decode_matches(inp, num_splits):
     o, lse = run_gpu(inp, num_splits)
     o_ref, lse_ref = reference(inp)
-    check_close(o, o_ref, BF16_MAX_ABS, BF16_MEAN_ABS, f"O (splits={num_splits})")
+    check_bf16(o, o_ref, f"O (splits={num_splits})")
     check_close(lse, lse_ref, LSE_ABS, None, f"LSE (splits={num_splits})")
     return o, lse
 
@@ -65,7 +65,7 @@ def case_inputs(case):
 def test_small(case, num_splits):
     inp, (o_ref, lse_ref) = case_inputs(case)
     o, lse = run_gpu(inp, num_splits)
-    check_close(o, o_ref, BF16_MAX_ABS, BF16_MEAN_ABS, "O")
+    check_bf16(o, o_ref, "O")
     check_close(lse, lse_ref, LSE_ABS, None, "LSE")
 
 
@@ -124,7 +124,7 @@ def test_caller_workspace_and_lse_optional():
     o = torch.empty_like(q)
     api.fa_decode_paged(q, kp, vp, bt, sl, S, o, None, inp.scale, ws)
     o_ref, _ = reference(inp)
-    check_close(to_np(o), o_ref, BF16_MAX_ABS, BF16_MEAN_ABS, "O with caller workspace")
+    check_bf16(to_np(o), o_ref, "O with caller workspace")
     # library-allocated (stream-ordered) workspace
     o2 = torch.empty_like(q)
     api.fa_decode_paged(q, kp, vp, bt, sl, S, o2, None, inp.scale, None)
@@ -158,5 +158,5 @@ def test_long_decode_full_size():
     o, lse = assert_decode_matches(inp, 0)
     o1, lse1 = run_gpu(inp, 1)  # one split walks the whole 131072-token context
     o_ref, lse_ref = reference(inp)
-    check_close(o1, o_ref, BF16_MAX_ABS, BF16_MEAN_ABS, "O one split")
+    check_bf16(o1, o_ref, "O one split")
     check_close(lse1, lse_ref, LSE_ABS, None, "LSE one split")
