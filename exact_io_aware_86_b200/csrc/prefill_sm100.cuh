@@ -56,8 +56,8 @@ constexpr int NUM_THREADS = NUM_WARPS * 32;
 // kRegsLaunch per thread; the control group gives most of its share to the
 // softmax groups: 128*kRegsControl + 256*kRegsSoftmax <= 384*kRegsLaunch.
 constexpr uint32_t kRegsLaunch = 168;
-constexpr uint32_t kRegsControl = 64;
-constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsControl = 96;
+constexpr uint32_t kRegsSoftmax = 200;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= NUM_THREADS * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t TMEM_COLS = 512;
@@ -288,6 +288,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           return true;
         };
         if (!issue_kv(min(2, 2 * nmax))) break;
+        if (it + 1 < num_items) {
+          // the next item's Q tiles come from DRAM; pull them into L2 now so
+          // their load at the next item boundary is short
+          const int2 nx = sh.items[it + 1];
+          int ns, nl;
+          seq_range(p, nx.x, ns, nl);
+          const int nq0 = ns + (nx.y >> 16) * ROWS_PER_ITEM, nh = nx.y & 0xFFFF;
+#pragma unroll
+          for (int t = 0; t < NQT; ++t)
+#pragma unroll
+            for (int pn = 0; pn < C::PANELS; ++pn)
+              tma_prefetch_l2_2d(&tmQ, nh * D + pn * 64, nq0 + t * BM);
+        }
         if (!mbar_wait(&sh.q_empty, (q_it & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&sh.q_full, NQT * C::TILE_BYTES);
 #pragma unroll
@@ -315,25 +328,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t kv_it = 0, q_it = 0;
       uint32_t p_phase0 = 0, p_phase1 = 0;
       bool ok = true;
+      // Descriptors of the first Q tile and the first K/V slot; every other
+      // operand is the same descriptor with its start address advanced.
+      const uint64_t q_desc = sdesc_sw128(q_addr, 16, 1024);           // K-major
+      const uint64_t k_desc = sdesc_sw128(kv_addr, 16, 1024);          // K-major
+      const uint64_t v_desc = sdesc_sw128(kv_addr, C::PANEL_BYTES, 1024);  // MN-major
       // O_t += P_t V   (A = P from TMEM, B = V, MN-major)
       auto issue_pv = [&](int t, uint32_t v_idx, bool first) {
-        const uint32_t v_base = kv_addr + (v_idx % C::STAGES) * C::TILE_BYTES;
+        const uint64_t vd = sdesc_advance(v_desc, (v_idx % C::STAGES) * C::TILE_BYTES);
+        const uint32_t d_tmem = tmem + 256 + t * 128, a_tmem = tmem + t * 128;
+        umma_ts(d_tmem, a_tmem, vd, C::IDESC_PV, first ? 0u : 1u);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(v_base + kk * 16 * 128, C::PANEL_BYTES, 1024);
-          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bdesc, C::IDESC_PV,
-                  (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 1; kk < BN / 16; ++kk)
+          umma_ts(d_tmem, a_tmem + kk * 8, sdesc_advance(vd, kk * 16 * 128), C::IDESC_PV, 1u);
       };
       // S_t = Q_t K^T   (both K-major)
       auto issue_s = [&](int t, uint32_t k_idx) {
-        const uint32_t a_base = q_addr + t * C::TILE_BYTES;
-        const uint32_t b_base = kv_addr + (k_idx % C::STAGES) * C::TILE_BYTES;
+        const uint64_t qd = sdesc_advance(q_desc, t * C::TILE_BYTES);
+        const uint64_t kd = sdesc_advance(k_desc, (k_idx % C::STAGES) * C::TILE_BYTES);
+        const uint32_t d_tmem = tmem + t * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + t * 128, sdesc_sw128(a_base + off, 16, 1024),
-                  sdesc_sw128(b_base + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+          umma_ss(d_tmem, sdesc_advance(qd, off), sdesc_advance(kd, off), C::IDESC_S,
+                  kk > 0 ? 1u : 0u);
         }
       };
       for (int it = 0; it < num_items && ok; ++it) {
@@ -425,7 +443,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // row sums, each as two interleaved fp32 pairs: le = exact sum of
       // exp (for the LSE), lr = sum of the bf16 values the PV MMA consumes
       // (normalises O consistently with its own weights)
-      uint64_t le_a = 0, le_b = 0, lr_a = 0, lr_b = 0;
+      uint64_t le_a = 0, le_b = 0;
+      float lr_a0 = 0.f, lr_a1 = 0.f, lr_b0 = 0.f, lr_b1 = 0.f;
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait(&sh.s_full[t], s_phase, abort)) { ok = false; break; }
         s_phase ^= 1;
@@ -467,8 +486,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t a2 = f2_pack(alpha, alpha);
           le_a = f2_mul(le_a, a2);
           le_b = f2_mul(le_b, a2);
-          lr_a = f2_mul(lr_a, a2);
-          lr_b = f2_mul(lr_b, a2);
+          lr_a0 *= alpha;
+          lr_a1 *= alpha;
+          lr_b0 *= alpha;
+          lr_b1 *= alpha;
           m_ref = m_new;
           rescale = true;
         }
@@ -492,14 +513,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             float p0, p1;
             f2_unpack(pr, p0, p1);
             const uint32_t pp = pack_bf16x2(p0, p1);
-            const uint64_t pq =
-                f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xFFFF0000u));
             if ((e >> 1) & 1) {
               le_b = f2_add(le_b, pr);
-              lr_b = f2_add(lr_b, pq);
+              lr_b0 = add_bf16lo_f32(pp, lr_b0);
+              lr_b1 = add_bf16hi_f32(pp, lr_b1);
             } else {
               le_a = f2_add(le_a, pr);
-              lr_a = f2_add(lr_a, pq);
+              lr_a0 = add_bf16lo_f32(pp, lr_a0);
+              lr_a1 = add_bf16hi_f32(pp, lr_a1);
             }
             s[c][e >> 1] = pp;
           }
@@ -536,9 +557,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       f2_unpack(le_a, la0, la1);
       f2_unpack(le_b, lb0, lb1);
       const float l_exact = (la0 + la1) + (lb0 + lb1);
-      f2_unpack(lr_a, la0, la1);
-      f2_unpack(lr_b, lb0, lb1);
-      const float l_round = (la0 + la1) + (lb0 + lb1);
+      const float l_round = (lr_a0 + lr_a1) + (lr_b0 + lr_b1);
       const bool valid = qpos < len;
       const float inv_l = 1.f / l_round;
       const size_t grow = (size_t)(start + qpos);
