@@ -45,6 +45,9 @@ def load_library(path: str = LIB_PATH):
     lib.fa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, i32]
     lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32, i32, i32,
                                     i32, f32, vp, vp, sz]
+    lib.fa_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32,
+                                            i32, i32, i32, f32, vp]
+    lib.fa_decode_paged_noalloc.restype = ctypes.c_int
     lib.fa_decode_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.fa_decode_workspace_size.restype = sz
     lib.fa_decode_auto_splits.argtypes = [i32, i32, i32, i32]
@@ -194,6 +197,26 @@ def fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int,
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), page_size,
         int(num_splits), _ptr(o), _stream(stream), B, Hq, Hkv, d, max_blocks, num_pages,
         float(scale), _ptr(lse), _ptr(workspace), ws_bytes), "fa_decode_paged")
+
+
+def fa_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, num_splits: int, o,
+                            lse=None, scale: float = 0.0, stream=None) -> None:
+    """Calls ``fa_decode_paged_noalloc``: the same decode as
+    ``fa_decode_paged``, with the split scratch taken from a fixed 16 MiB
+    array inside the library, for callers that cannot allocate device memory
+    at decode time.  Raises FAError(FA_ERR_UNSUPPORTED) when the split scratch
+    this shape needs is larger than that array.  Concurrent calls on
+    different streams share the array and must not overlap.
+    """
+    B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
+        q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16)
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    _check(load_library().fa_decode_paged_noalloc(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), page_size,
+        int(num_splits), _ptr(o), _stream(stream), B, Hq, Hkv, d, max_blocks, num_pages,
+        float(scale), _ptr(lse)), "fa_decode_paged_noalloc")
 
 
 def decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int = 0,

@@ -347,3 +347,60 @@ const char* fa_get_error_string(fa_status status) {
 int fa_version(void) { return 100; }
 
 }  // extern "C"
+
+// --------------------------------------------------------------------------
+// Paged decode without any allocation (fa_decode_paged_noalloc).
+//
+// Some callers cannot allocate device memory at the point where they run a
+// decode step: a serving engine that has already handed nearly all of HBM to
+// its KV-cache pool, or a step loop that must not block in, or fail inside,
+// the allocator once it is running.  This entry point takes its split
+// scratch from a fixed array compiled into the library instead.  Every GPU
+// that loads the library holds the array until the process exits.
+// --------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_decode_scratch on the current device.  The first call
+// on each device looks it up (cudaGetSymbolAddress with that device current)
+// and caches it; later calls only read the cache.
+void* decode_scratch_on_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return nullptr;
+    addr[dev] = ptr;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" fa_status fa_decode_paged_noalloc(const void* q, const void* k_pages,
+                                             const void* v_pages, const int32_t* block_table,
+                                             const int32_t* seq_lens, int page_size,
+                                             int num_splits, void* o, fa_stream_t stream, int B,
+                                             int Hq, int Hkv, int d, int max_blocks_per_seq,
+                                             int num_pages, float scale, float* lse) {
+  if (num_splits < 0 || B < 0 || Hq <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  const int S = num_splits == 0 ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, 0) : num_splits;
+  const size_t need = fa_decode_workspace_size(B, Hq, d, S);
+  if (need > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (need > 0) {
+    scratch = decode_scratch_on_current_device();
+    if (!scratch) return FA_ERR_CUDA;
+  }
+  return fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, page_size, S, o, stream, B,
+                         Hq, Hkv, d, max_blocks_per_seq, num_pages, scale, lse, scratch,
+                         need > 0 ? kNoAllocScratchBytes : 0);
+}

@@ -112,6 +112,33 @@ fa_status fa_decode_paged(const void *q, const void *k_pages, const void *v_page
                           int d, int max_blocks_per_seq, int num_pages, float scale, float *lse,
                           void *workspace, size_t workspace_bytes);
 
+/*
+ * Paged decode that allocates nothing (no counterpart in the pages; this is
+ * a deployment convenience).  Same arguments and result as fa_decode_paged
+ * without the workspace pair: the split scratch comes from a 16 MiB array
+ * compiled into the library, held by every GPU that loads it until exit.
+ *
+ * For callers that cannot allocate device memory when they run a decode
+ * step, e.g. a serving engine that has already reserved nearly all of HBM
+ * for its KV-cache pool, or a step loop that must not block in or fail
+ * inside an allocator.
+ *
+ *   - Returns FA_ERR_UNSUPPORTED, launching nothing, when
+ *     fa_decode_workspace_size(B, Hq, d, resolved num_splits) exceeds
+ *     16 MiB; use fewer splits or fa_decode_paged with your own workspace.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (nothing in it needs to start at zero).  Calls that overlap on the GPU
+ *     (different streams without ordering between them) race on it.
+ */
+fa_status fa_decode_paged_noalloc(const void *q, const void *k_pages, const void *v_pages,
+                                  const int32_t *block_table, const int32_t *seq_lens,
+                                  int page_size, int num_splits, void *o, fa_stream_t stream,
+                                  int B, int Hq, int Hkv, int d, int max_blocks_per_seq,
+                                  int num_pages, float scale, float *lse);
+
 /* Bytes of workspace fa_decode_paged needs for this shape and split count
  * (partial outputs fp32 [B, Hq, S, d] and partial LSEs fp32 [B, Hq, S]). */
 size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits);
