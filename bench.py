@@ -296,7 +296,10 @@ class DeviceWorkload:
         if din is not None:
             self.dq, self.kp, self.vp = (t.to(dev) for t in (din.q, din.k_pages, din.v_pages))
             self.bt, self.sl = din.block_table.to(dev), din.seq_lens.to(dev)
-            self.splits = api.decode_auto_splits(din.B, din.Hkv, din.block_table.shape[1])
+            # automatic page ranges (num_splits = 0); splits = the most ranges a
+            # request can get, which sizes the workspace
+            self.splits = api.decode_auto_splits(din.B, din.Hkv, din.block_table.shape[1],
+                                                 din.page_size)
             nbytes = api.decode_workspace_size(din.B, din.Hq, din.d, self.splits)
             self.ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) if nbytes else None
             self.do = torch.empty_like(self.dq)
@@ -305,7 +308,7 @@ class DeviceWorkload:
     def launches_per_step(self):
         n = 1 if self.pin is not None else 0
         if self.din is not None:
-            n += 1 + (1 if self.splits > 1 else 0)
+            n += 1 + (2 if self.splits > 1 else 0)  # split kernel (+ plan and combine)
         return n
 
     def prefill(self):
@@ -313,7 +316,7 @@ class DeviceWorkload:
                        self.pin.scale, self.max_len)
 
     def decode(self):
-        api.fa_decode_paged(self.dq, self.kp, self.vp, self.bt, self.sl, self.splits, self.do,
+        api.fa_decode_paged(self.dq, self.kp, self.vp, self.bt, self.sl, 0, self.do,
                             self.dlse, self.din.scale, self.ws)
 
 
@@ -457,11 +460,11 @@ def run_gpu(args, world, rank, local):
         parts["decode"] = {
             "workload": din.name, "value": round(gbs, 1), "unit": "GB/s",
             "ms": round(dec_ms, 4), "ms_min": round(min(dec), 4), "bytes": by,
-            "num_splits": w.splits,
+            "max_ranges_per_request": w.splits,
             "workspace_bytes": api.decode_workspace_size(din.B, din.Hq, din.d, w.splits),
             "roofline": roofline("decode", gbs / world, peaks["hbm_gbs"], "GB/s",
                                  dram_traffic("decode", din.name)),
-            "launches_per_call": 1 + (1 if w.splits > 1 else 0),
+            "launches_per_call": 1 + (2 if w.splits > 1 else 0),
         }
     head = parts.get("prefill") or parts.get("decode")
     dominant = max(parts.values(), key=lambda p: p["ms"])

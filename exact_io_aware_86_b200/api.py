@@ -50,7 +50,7 @@ def load_library(path: str = LIB_PATH):
     lib.fa_decode_paged_noalloc.restype = ctypes.c_int
     lib.fa_decode_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.fa_decode_workspace_size.restype = sz
-    lib.fa_decode_auto_splits.argtypes = [i32, i32, i32, i32]
+    lib.fa_decode_auto_splits.argtypes = [i32, i32, i32, i32, i32]
     lib.fa_prefill_f32.argtypes = lib.fa_prefill.argtypes
     lib.fa_decode_paged_f32.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
                                         i32, f32, vp]
@@ -154,8 +154,11 @@ def decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:
     return int(load_library().fa_decode_workspace_size(B, Hq, d, num_splits))
 
 
-def decode_auto_splits(B: int, Hkv: int, max_blocks_per_seq: int, num_sms: int = 0) -> int:
-    return int(load_library().fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, num_sms))
+def decode_auto_splits(B: int, Hkv: int, max_blocks_per_seq: int, page_size: int,
+                       num_sms: int = 0) -> int:
+    """The split count ``num_splits = 0`` resolves to (sizes the workspace)."""
+    return int(load_library().fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, page_size,
+                                                    num_sms))
 
 
 def _decode_shapes(q, k_pages, v_pages, block_table, seq_lens, dt):
@@ -202,7 +205,7 @@ def fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int,
 def fa_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, num_splits: int, o,
                             lse=None, scale: float = 0.0, stream=None) -> None:
     """Calls ``fa_decode_paged_noalloc``: the same decode as
-    ``fa_decode_paged``, with the split scratch taken from a fixed 16 MiB
+    ``fa_decode_paged``, with the split scratch taken from a fixed 64 MiB
     array inside the library, for callers that cannot allocate device memory
     at decode time.  Raises FAError(FA_ERR_UNSUPPORTED) when the split scratch
     this shape needs is larger than that array.  Concurrent calls on
@@ -225,12 +228,13 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int = 0
     ``fa_decode_paged``.  Returns (o, lse or None)."""
     B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
         q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16)
-    S = num_splits if num_splits > 0 else decode_auto_splits(B, Hkv, max_blocks)
+    S = num_splits if num_splits > 0 else decode_auto_splits(B, Hkv, max_blocks, page_size)
     o = torch.empty_like(q)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if return_lse else None
     nbytes = decode_workspace_size(B, Hq, d, S)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device) if nbytes else None
-    fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, S, o, lse, scale, ws, stream)
+    fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits, o, lse, scale, ws,
+                    stream)
     return o, lse
 
 

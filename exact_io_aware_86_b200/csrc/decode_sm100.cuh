@@ -10,21 +10,28 @@
 // KV cache block by block and lets the online softmax do the reduction, on
 // non-contiguous pages without copying them into a contiguous tensor):
 //
-//   D1 (split kernel): one CTA per (split, group of up to 8 kv heads,
-//   request).  A producer warp gathers the split's pages 16 tokens at a time
+//   Plan: a one-CTA kernel counts each request's page ranges (device-side
+//   seq_lens) and writes their prefix sums, so the split kernel can walk a
+//   flat list of non-empty ranges (the pages' Plan-Run split of scheduling
+//   and execution, "gsyq.cn FA vs FIA" section 2).
+//
+//   D1 (split kernel): persistent, one CTA per SM; CTA c takes ranges c,
+//   c + #CTAs, ... of the flat list (each for a group of up to 8 kv heads).
+//   A producer warp gathers each range's pages 16 tokens at a time
 //   into a shared-memory ring with TMA (3-D tensor maps over the pool with
 //   128-byte swizzle, one 16-token box per kv head and 64-wide half of
 //   head_dim; page_size is a multiple of 16).  Each consumer warp owns one kv head and the Hq/Hkv <= 8 query
 //   heads that read it, so every K/V byte is read from HBM once for the whole
 //   group.  Scores and the P V product use warp-level bf16 tensor-core MMAs
 //   (S^T = K Q^T with tokens as rows, O^T += V^T P^T); the online softmax
-//   keeps a running max and sum per query head.  The split writes its
-//   normalised partial O and its LSE (fp32) to the workspace, or, with one
-//   split, the final bf16 O and LSE directly.
+//   keeps a running max and sum per query head.  A range writes its
+//   normalised partial O and its LSE (fp32) to the workspace, or, when it is
+//   its request's only range, the final bf16 O and LSE directly.  In the
+//   automatic mode every range spans the same number of pages, so the flat
+//   list is made of near-equal items and the CTAs finish together.
 //
 //   D2 (combine): per (request, query head), LSE = log sum_s exp(lse_s) and
-//   O = sum_s exp(lse_s - LSE) O_s; splits with no tokens have lse = -inf and
-//   weigh zero.
+//   O = sum_s exp(lse_s - LSE) O_s over the request's ranges.
 #pragma once
 
 #include "ptx.cuh"
@@ -41,13 +48,16 @@ struct Params {
   const __nv_bfloat16* q;     // [B, Hq, D]
   const int32_t* block_table; // [B, max_blocks]
   const int32_t* seq_lens;    // [B]
-  float* o_part;              // [B, Hq, S, D]  (num_splits > 1)
-  float* lse_part;            // [B, Hq, S]
-  __nv_bfloat16* o;           // [B, Hq, D]     (num_splits == 1)
+  const int32_t* split_prefix;  // [B+1] exclusive prefix of per-request range counts, or null
+  float* o_part;              // [B, Hq, s_max, D]   partial outputs (normalised)
+  float* lse_part;            // [B, Hq, s_max]      partial LSEs
+  __nv_bfloat16* o;           // [B, Hq, D]
   float* lse;                 // [B, Hq] or null
-  int B, Hq, Hkv, group, hpb;
-  int page_size, max_blocks, num_pages, num_splits;
-  int half_bytes;             // bytes of the K (or V) part of one stage
+  int B, Hq, Hkv, group, hpb, ngroups;
+  int page_size, max_blocks, num_pages;
+  int s_max;        // partial slots per (request, head)
+  int chunk_pages;  // > 0: every range spans chunk_pages pages; 0: s_max near-equal ranges per request
+  int half_bytes;   // bytes of the K (or V) part of one stage
   float scale_log2;
 };
 
@@ -70,6 +80,110 @@ __device__ __forceinline__ uint32_t kv_off(int hpb, int panel, int hh, int tok, 
   return (uint32_t)((panel * hpb + hh) * BOX_BYTES + tok * 128 + ((ch ^ (tok & 7)) << 4));
 }
 
+// Context length of request b as the kernels use it (out-of-range values are
+// a bounds error and are clamped), and its page count.
+__device__ __forceinline__ int request_pages(const Params& p, int b, int& seq, bool report) {
+  seq = __ldg(p.seq_lens + b);
+  const int cap = p.max_blocks * p.page_size;
+  if (seq < 0 || seq > cap) {
+    if (report) report_error(kDevErrBounds);
+    seq = seq < 0 ? 0 : cap;
+  }
+  return (seq + p.page_size - 1) / p.page_size;
+}
+
+// Pages per range and number of non-empty ranges of a request.
+__device__ __forceinline__ int range_pages(const Params& p, int npages) {
+  return p.chunk_pages > 0 ? p.chunk_pages : (npages + p.s_max - 1) / p.s_max;
+}
+__device__ __forceinline__ int num_ranges(const Params& p, int npages) {
+  if (npages <= 0) return 0;
+  const int c = range_pages(p, npages);
+  return (npages + c - 1) / c;
+}
+
+// Plan: exclusive prefix sums of the per-request range counts (one CTA of
+// 1024 threads, requests in chunks of 1024).
+__global__ void __launch_bounds__(1024) plan_kernel(const Params p, int32_t* __restrict__ prefix) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < p.B; base += 1024) {
+    const int b = base + tid;
+    int n = 0;
+    if (b < p.B) {
+      int seq;
+      n = num_ranges(p, request_pages(p, b, seq, true));
+    }
+    int x = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_sums[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += y;
+      }
+      warp_sums[lane] = w;
+    }
+    __syncthreads();
+    const int incl = carry + x + (warp > 0 ? warp_sums[warp - 1] : 0);
+    if (b < p.B) prefix[b] = incl - n;
+    __syncthreads();
+    if (tid == 1023) carry = incl;
+    __syncthreads();
+  }
+  if (tid == 0) prefix[p.B] = carry;
+}
+
+// Work item i -> (request b, range s, kv-head group y); items are the
+// non-empty ranges of every request, kv-head groups fastest.
+__device__ __forceinline__ void item_of(const Params& p, int i, int& b, int& s, int& y) {
+  y = i % p.ngroups;
+  const int bs = i / p.ngroups;
+  if (!p.split_prefix) {
+    b = bs;
+    s = 0;
+    return;
+  }
+  int lo = 0, hi = p.B - 1;  // last b with prefix[b] <= bs
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.split_prefix + mid) <= bs) lo = mid; else hi = mid - 1;
+  }
+  b = lo;
+  s = bs - __ldg(p.split_prefix + lo);
+}
+
+// Token range [tok_begin, tok_end) of range s of request b.
+__device__ __forceinline__ void item_tokens(const Params& p, int b, int s, int& tok_begin,
+                                            int& tok_end, int& nranges) {
+  int seq;
+  // the plan kernel reports bad lengths when there is a plan; otherwise here
+  const int npages = request_pages(p, b, seq, !p.split_prefix);
+  if (!p.split_prefix) {
+    tok_begin = 0;
+    tok_end = seq;
+    nranges = 1;
+    return;
+  }
+  const int c = range_pages(p, npages);
+  const int pg0 = min(npages, s * c), pg1 = min(npages, pg0 + c);
+  tok_begin = pg0 * p.page_size;
+  tok_end = min(seq, pg1 * p.page_size);
+  nranges = num_ranges(p, npages);
+}
+
+// Persistent: CTA c takes items c, c + gridDim.x, ...; the TMA ring runs on
+// across item boundaries.
 template <int D>
 __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
     split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -84,9 +198,6 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
   int* abort_flag = reinterpret_cast<int*>(empty + STAGES);
   volatile int* abort = abort_flag;
 
-  const int split = blockIdx.x;
-  const int kvh0 = blockIdx.y * p.hpb;
-  const int b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
   const int nconsumers = p.hpb;
 
@@ -100,264 +211,310 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
   }
   __syncthreads();
 
-  // The split's token range: pages [p0, p1) of this request.
-  int seq = __ldg(p.seq_lens + b);
-  if (seq < 0 || seq > p.max_blocks * p.page_size) {
-    if (threadIdx.x == 0) report_error(kDevErrBounds);
-    seq = seq < 0 ? 0 : p.max_blocks * p.page_size;
-  }
-  const int npages = (seq + p.page_size - 1) / p.page_size;
-  const int chunk = (npages + p.num_splits - 1) / p.num_splits;
-  const int pg0 = min(npages, split * chunk);
-  const int pg1 = min(npages, pg0 + chunk);
-  const int tok_begin = pg0 * p.page_size;
-  const int tok_end = min(seq, pg1 * p.page_size);
-  const int nstages = tok_end > tok_begin ? (tok_end - tok_begin + TOK - 1) / TOK : 0;
+  const int total = (p.split_prefix ? __ldg(p.split_prefix + p.B) : p.B) * p.ngroups;
 
   if (warp == nconsumers) {
     // ======================= producer =======================
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int32_t* bt = p.block_table + (size_t)b * p.max_blocks;
-      int st = 0;
-      for (; st < nstages; ++st) {
-        const int slot = st % STAGES;
-        if (!mbar_wait(&empty[slot], ((st / STAGES) & 1) ^ 1, abort)) break;
-        // page_size is a multiple of TOK, so a stage never crosses a page
-        const int t0 = tok_begin + st * TOK;
-        const int page = __ldg(bt + t0 / p.page_size);
-        int z;
-        if (page < 0 || page >= p.num_pages) {
-          report_error(kDevErrBounds);
-          z = -TOK;  // whole box outside the pool: TMA fills zeros
-        } else {
-          z = page * p.page_size + (t0 % p.page_size);
-        }
-        mbar_arrive_expect_tx(&full[slot], 2 * p.half_bytes);
-        uint8_t* kdst = smem + slot * sbytes;
-        uint8_t* vdst = kdst + p.half_bytes;
-        for (int pn = 0; pn < C::PANELS; ++pn)
-          for (int hh = 0; hh < p.hpb; ++hh) {
-            const int off = (pn * p.hpb + hh) * BOX_BYTES;
-            tma_load_3d(kdst + off, &tmK, &full[slot], pn * 64, kvh0 + hh, z);
-            tma_load_3d(vdst + off, &tmV, &full[slot], pn * 64, kvh0 + hh, z);
+      int g = 0;  // stages issued so far (ring position)
+      bool ok = true;
+      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        int b, s, y, tb, te, nr;
+        item_of(p, i, b, s, y);
+        item_tokens(p, b, s, tb, te, nr);
+        const int kvh0 = y * p.hpb;
+        const int32_t* bt = p.block_table + (size_t)b * p.max_blocks;
+        const int nst = te > tb ? (te - tb + TOK - 1) / TOK : 0;
+        for (int st = 0; st < nst; ++st, ++g) {
+          const int slot = g % STAGES;
+          if (!mbar_wait(&empty[slot], ((g / STAGES) & 1) ^ 1, abort)) { ok = false; break; }
+          // page_size is a multiple of TOK, so a stage never crosses a page
+          const int t0 = tb + st * TOK;
+          const int page = __ldg(bt + t0 / p.page_size);
+          int z;
+          if (page < 0 || page >= p.num_pages) {
+            report_error(kDevErrBounds);
+            z = -TOK;  // whole box outside the pool: TMA fills zeros
+          } else {
+            z = page * p.page_size + (t0 % p.page_size);
           }
+          mbar_arrive_expect_tx(&full[slot], 2 * p.half_bytes);
+          uint8_t* kdst = smem + slot * sbytes;
+          uint8_t* vdst = kdst + p.half_bytes;
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            for (int hh = 0; hh < p.hpb; ++hh) {
+              const int off = (pn * p.hpb + hh) * BOX_BYTES;
+              tma_load_3d(kdst + off, &tmK, &full[slot], pn * 64, kvh0 + hh, z);
+              tma_load_3d(vdst + off, &tmV, &full[slot], pn * 64, kvh0 + hh, z);
+            }
+        }
       }
       // every load issued must land before the CTA exits
-      for (int s = 0; s < STAGES && s < st; ++s) {
-        const int last = st - 1 - ((st - 1 - s) % STAGES);
+      for (int s = 0; s < STAGES && s < g; ++s) {
+        const int last = g - 1 - ((g - 1 - s) % STAGES);
         mbar_wait_bounded(&full[last % STAGES], (last / STAGES) & 1);
       }
     }
   } else {
     // ======================= consumers: one warp per kv head =======================
     const int hh = warp;
-    const int kvh = kvh0 + hh;
-    const int g = lane >> 2, tq = lane & 3;
-    // Q^T fragments (MMA B operand, k = head_dim, n = query head of the group)
-    uint32_t qb0[C::KS], qb1[C::KS];
-    {
-      const bool real = g < p.group;
-      const __nv_bfloat16* qrow = p.q + ((size_t)b * p.Hq + (size_t)kvh * p.group + (real ? g : 0)) * D;
-#pragma unroll
-      for (int ks = 0; ks < C::KS; ++ks) {
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * tq);
-        qb0[ks] = real ? __ldg(w) : 0u;
-        qb1[ks] = real ? __ldg(w + 4) : 0u;
-      }
-    }
-    float acc[C::KS][4];
-#pragma unroll
-    for (int mt = 0; mt < C::KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-    // query heads 2tq, 2tq+1: running max, exact sum of exp (for the LSE) and
-    // sum of the bf16-rounded weights the PV MMA uses (normalises O)
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
+    const int g8 = lane >> 2, tq = lane & 3;
     const float sl = p.scale_log2;
     const uint32_t sbase = smem_u32(smem);
-
-    // ldmatrix row/chunk assignment of this lane
-    const int lm = lane >> 3, lr = lane & 7;
-    for (int st = 0; st < nstages; ++st) {
-      const int slot = st % STAGES;
-      if (!mbar_wait(&full[slot], (st / STAGES) & 1, abort)) break;
-      const uint32_t kb = sbase + slot * sbytes;
-      const uint32_t vb = kb + p.half_bytes;
-      const int valid = min(TOK, tok_end - (tok_begin + st * TOK));
-      if (valid < TOK) {
-        // V rows past the context are not part of the sum; their P is zero,
-        // but 0 * (garbage) may be NaN, so clear them for this warp's head.
-        uint8_t* vgen = smem + slot * sbytes + p.half_bytes;
-        for (int idx = lane; idx < (TOK - valid) * C::PANELS * 8; idx += 32) {
-          const int tok = valid + idx / (C::PANELS * 8);
-          const int rem = idx % (C::PANELS * 8);
-          *reinterpret_cast<uint4*>(vgen + kv_off(p.hpb, rem / 8, hh, tok, rem % 8)) =
-              make_uint4(0, 0, 0, 0);
-        }
-        __syncwarp();
-      }
-      // ---- S^T[tok][n] = sum_d K[tok][d] Q[n][d] ----
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
+    const int lm = lane >> 3, lr = lane & 7;  // ldmatrix row/chunk assignment of this lane
+    int g = 0;  // stages consumed so far (ring position)
+    bool ok = true;
+    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+      int b, s, y, tb, te, nr;
+      item_of(p, i, b, s, y);
+      item_tokens(p, b, s, tb, te, nr);
+      const int kvh = y * p.hpb + hh;
+      const int nst = te > tb ? (te - tb + TOK - 1) / TOK : 0;
+      // Q^T fragments (MMA B operand, k = head_dim, n = query head of the group)
+      uint32_t qb0[C::KS], qb1[C::KS];
+      {
+        const bool real = g8 < p.group;
+        const __nv_bfloat16* qrow =
+            p.q + ((size_t)b * p.Hq + (size_t)kvh * p.group + (real ? g8 : 0)) * D;
 #pragma unroll
-      for (int ks = 0; ks < C::KS; ++ks) {
-        // matrices: 0 = tok 0-7 / d lo, 1 = tok 8-15 / d lo, 2 = tok 0-7 / d hi, 3 = tok 8-15 / d hi
-        const int tok = lr + ((lm & 1) << 3);
-        const int d0 = ks * 16 + ((lm >> 1) << 3);
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(kb + kv_off(p.hpb, d0 >> 6, hh, tok, (d0 & 63) >> 3), a0, a1, a2, a3);
-        mma_bf16_16816(c, a0, a1, a2, a3, qb0[ks], qb1[ks]);
+        for (int ks = 0; ks < C::KS; ++ks) {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * tq);
+          qb0[ks] = real ? __ldg(w) : 0u;
+          qb1[ks] = real ? __ldg(w + 4) : 0u;
+        }
       }
-      // rows: token g (c0, c1) and g + 8 (c2, c3); columns: query heads 2tq, 2tq+1
-      float s00 = c[0] * sl, s01 = c[1] * sl, s10 = c[2] * sl, s11 = c[3] * sl;
-      if (g >= valid) s00 = s01 = -INFINITY;
-      if (g + 8 >= valid) s10 = s11 = -INFINITY;
-      float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+      float acc[C::KS][4];
+#pragma unroll
+      for (int mt = 0; mt < C::KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      // query heads 2tq, 2tq+1: running max, exact sum of exp (for the LSE) and
+      // sum of the bf16-rounded weights the PV MMA uses (normalises O)
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
+      for (int st = 0; st < nst; ++st, ++g) {
+        const int slot = g % STAGES;
+        if (!mbar_wait(&full[slot], (g / STAGES) & 1, abort)) { ok = false; break; }
+        const uint32_t kb = sbase + slot * sbytes;
+        const uint32_t vb = kb + p.half_bytes;
+        const int valid = min(TOK, te - (tb + st * TOK));
+        if (valid < TOK) {
+          // V rows past the context are not part of the sum; their P is zero,
+          // but 0 * (garbage) may be NaN, so clear them for this warp's head.
+          uint8_t* vgen = smem + slot * sbytes + p.half_bytes;
+          for (int idx = lane; idx < (TOK - valid) * C::PANELS * 8; idx += 32) {
+            const int tok = valid + idx / (C::PANELS * 8);
+            const int rem = idx % (C::PANELS * 8);
+            *reinterpret_cast<uint4*>(vgen + kv_off(p.hpb, rem / 8, hh, tok, rem % 8)) =
+                make_uint4(0, 0, 0, 0);
+          }
+          __syncwarp();
+        }
+        // ---- S^T[tok][n] = sum_d K[tok][d] Q[n][d] ----
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ++ks) {
+          // matrices: 0 = tok 0-7 / d lo, 1 = tok 8-15 / d lo, 2 = tok 0-7 / d hi, 3 = tok 8-15 / d hi
+          const int tok = lr + ((lm & 1) << 3);
+          const int d0 = ks * 16 + ((lm >> 1) << 3);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(kb + kv_off(p.hpb, d0 >> 6, hh, tok, (d0 & 63) >> 3), a0, a1, a2, a3);
+          mma_bf16_16816(c, a0, a1, a2, a3, qb0[ks], qb1[ks]);
+        }
+        // rows: token g8 (c0, c1) and g8 + 8 (c2, c3); columns: query heads 2tq, 2tq+1
+        float s00 = c[0] * sl, s01 = c[1] * sl, s10 = c[2] * sl, s11 = c[3] * sl;
+        if (g8 >= valid) s00 = s01 = -INFINITY;
+        if (g8 + 8 >= valid) s10 = s11 = -INFINITY;
+        float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: valid >= 1
+        const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);    // ex2(-inf) = 0
+        const float p00 = ex2(s00 - mn0), p01 = ex2(s01 - mn1);
+        const float p10 = ex2(s10 - mn0), p11 = ex2(s11 - mn1);
+        // P^T in bf16 (the MMA operand); the row sums use the same rounded values
+        const uint32_t x0 = pack_bf16x2(p00, p01), x1 = pack_bf16x2(p10, p11);
+        l0 = l0 * al0 + (p00 + p10);
+        l1 = l1 * al1 + (p01 + p11);
+        r0 = r0 * al0 + (__uint_as_float(x0 << 16) + __uint_as_float(x1 << 16));
+        r1 = r1 * al1 + (__uint_as_float(x0 & 0xFFFF0000u) + __uint_as_float(x1 & 0xFFFF0000u));
+        m0 = mn0;
+        m1 = mn1;
+#pragma unroll
+        for (int mt = 0; mt < C::KS; ++mt) {
+          acc[mt][0] *= al0;
+          acc[mt][1] *= al1;
+          acc[mt][2] *= al0;
+          acc[mt][3] *= al1;
+        }
+        // P^T as the MMA B operand (k = token, n = query head)
+        const uint32_t pb0 = movmatrix_trans(x0);
+        const uint32_t pb1 = movmatrix_trans(x1);
+        // ---- O^T[d][n] += sum_tok V[tok][d] P[n][tok] ----
+#pragma unroll
+        for (int mt = 0; mt < C::KS; ++mt) {
+          // matrices: 0 = tok 0-7 / d lo, 1 = tok 0-7 / d hi, 2 = tok 8-15 / d lo, 3 = tok 8-15 / d hi
+          const int tok = lr + ((lm >> 1) << 3);
+          const int d0 = mt * 16 + ((lm & 1) << 3);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4_trans(vb + kv_off(p.hpb, d0 >> 6, hh, tok, (d0 & 63) >> 3), a0, a1, a2, a3);
+          mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+        }
+        if (valid < TOK) fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+      }
+      if (!ok) break;
+      // ---- finish: row sums over the 8 token lanes, normalise, write ----
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+        r0 += __shfl_xor_sync(0xffffffffu, r0, off);
+        r1 += __shfl_xor_sync(0xffffffffu, r1, off);
       }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: valid >= 1
-      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);    // ex2(-inf) = 0
-      const float p00 = ex2(s00 - mn0), p01 = ex2(s01 - mn1);
-      const float p10 = ex2(s10 - mn0), p11 = ex2(s11 - mn1);
-      // P^T in bf16 (the MMA operand); the row sums use the same rounded values
-      const uint32_t x0 = pack_bf16x2(p00, p01), x1 = pack_bf16x2(p10, p11);
-      l0 = l0 * al0 + (p00 + p10);
-      l1 = l1 * al1 + (p01 + p11);
-      r0 = r0 * al0 + (__uint_as_float(x0 << 16) + __uint_as_float(x1 << 16));
-      r1 = r1 * al1 + (__uint_as_float(x0 & 0xFFFF0000u) + __uint_as_float(x1 & 0xFFFF0000u));
-      m0 = mn0;
-      m1 = mn1;
+      const float inv0 = r0 > 0.f ? 1.f / r0 : 0.f, inv1 = r1 > 0.f ? 1.f / r1 : 0.f;
+      const float ln2 = 0.69314718055994531f;
+      const float lse0 = l0 > 0.f ? (m0 + __log2f(l0)) * ln2 : -INFINITY;
+      const float lse1 = l1 > 0.f ? (m1 + __log2f(l1)) * ln2 : -INFINITY;
+      const int n0 = 2 * tq, n1 = 2 * tq + 1;
+      const size_t head0 = (size_t)b * p.Hq + (size_t)kvh * p.group;
+      if (nr > 1) {
+        const int S = p.s_max;
 #pragma unroll
-      for (int mt = 0; mt < C::KS; ++mt) {
-        acc[mt][0] *= al0;
-        acc[mt][1] *= al1;
-        acc[mt][2] *= al0;
-        acc[mt][3] *= al1;
-      }
-      // P^T as the MMA B operand (k = token, n = query head)
-      const uint32_t pb0 = movmatrix_trans(x0);
-      const uint32_t pb1 = movmatrix_trans(x1);
-      // ---- O^T[d][n] += sum_tok V[tok][d] P[n][tok] ----
-#pragma unroll
-      for (int mt = 0; mt < C::KS; ++mt) {
-        // matrices: 0 = tok 0-7 / d lo, 1 = tok 0-7 / d hi, 2 = tok 8-15 / d lo, 3 = tok 8-15 / d hi
-        const int tok = lr + ((lm >> 1) << 3);
-        const int d0 = mt * 16 + ((lm & 1) << 3);
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4_trans(vb + kv_off(p.hpb, d0 >> 6, hh, tok, (d0 & 63) >> 3), a0, a1, a2, a3);
-        mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
-      }
-      if (valid < TOK) fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
-    }
-    // ---- finish: row sums over the 8 token lanes, normalise, write ----
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-      r0 += __shfl_xor_sync(0xffffffffu, r0, off);
-      r1 += __shfl_xor_sync(0xffffffffu, r1, off);
-    }
-    const float inv0 = r0 > 0.f ? 1.f / r0 : 0.f, inv1 = r1 > 0.f ? 1.f / r1 : 0.f;
-    const float ln2 = 0.69314718055994531f;
-    const float lse0 = l0 > 0.f ? (m0 + __log2f(l0)) * ln2 : -INFINITY;
-    const float lse1 = l1 > 0.f ? (m1 + __log2f(l1)) * ln2 : -INFINITY;
-    const int n0 = 2 * tq, n1 = 2 * tq + 1;
-    const size_t head0 = (size_t)b * p.Hq + (size_t)kvh * p.group;
-    if (p.num_splits > 1) {
-      const int S = p.num_splits;
-#pragma unroll
-      for (int mt = 0; mt < C::KS; ++mt) {
-        const int d = mt * 16 + g;
-        if (n0 < p.group) {
-          float* dst = p.o_part + ((head0 + n0) * S + split) * D;
-          dst[d] = acc[mt][0] * inv0;
-          dst[d + 8] = acc[mt][2] * inv0;
+        for (int mt = 0; mt < C::KS; ++mt) {
+          const int d = mt * 16 + g8;
+          if (n0 < p.group) {
+            float* dst = p.o_part + ((head0 + n0) * S + s) * D;
+            dst[d] = acc[mt][0] * inv0;
+            dst[d + 8] = acc[mt][2] * inv0;
+          }
+          if (n1 < p.group) {
+            float* dst = p.o_part + ((head0 + n1) * S + s) * D;
+            dst[d] = acc[mt][1] * inv1;
+            dst[d + 8] = acc[mt][3] * inv1;
+          }
         }
-        if (n1 < p.group) {
-          float* dst = p.o_part + ((head0 + n1) * S + split) * D;
-          dst[d] = acc[mt][1] * inv1;
-          dst[d + 8] = acc[mt][3] * inv1;
+        if (g8 == 0) {
+          if (n0 < p.group) p.lse_part[(head0 + n0) * S + s] = lse0;
+          if (n1 < p.group) p.lse_part[(head0 + n1) * S + s] = lse1;
         }
-      }
-      if (g == 0) {
-        if (n0 < p.group) p.lse_part[(head0 + n0) * S + split] = lse0;
-        if (n1 < p.group) p.lse_part[(head0 + n1) * S + split] = lse1;
-      }
-    } else {
+      } else {
+        // the request's only range (or an empty request with no plan): final output
 #pragma unroll
-      for (int mt = 0; mt < C::KS; ++mt) {
-        const int d = mt * 16 + g;
-        if (n0 < p.group) {
-          __nv_bfloat16* dst = p.o + (head0 + n0) * D;
-          dst[d] = __float2bfloat16_rn(acc[mt][0] * inv0);
-          dst[d + 8] = __float2bfloat16_rn(acc[mt][2] * inv0);
+        for (int mt = 0; mt < C::KS; ++mt) {
+          const int d = mt * 16 + g8;
+          if (n0 < p.group) {
+            __nv_bfloat16* dst = p.o + (head0 + n0) * D;
+            dst[d] = __float2bfloat16_rn(acc[mt][0] * inv0);
+            dst[d + 8] = __float2bfloat16_rn(acc[mt][2] * inv0);
+          }
+          if (n1 < p.group) {
+            __nv_bfloat16* dst = p.o + (head0 + n1) * D;
+            dst[d] = __float2bfloat16_rn(acc[mt][1] * inv1);
+            dst[d + 8] = __float2bfloat16_rn(acc[mt][3] * inv1);
+          }
         }
-        if (n1 < p.group) {
-          __nv_bfloat16* dst = p.o + (head0 + n1) * D;
-          dst[d] = __float2bfloat16_rn(acc[mt][1] * inv1);
-          dst[d + 8] = __float2bfloat16_rn(acc[mt][3] * inv1);
+        if (g8 == 0 && p.lse) {
+          if (n0 < p.group) p.lse[head0 + n0] = lse0;
+          if (n1 < p.group) p.lse[head0 + n1] = lse1;
         }
-      }
-      if (g == 0 && p.lse) {
-        if (n0 < p.group) p.lse[head0 + n0] = lse0;
-        if (n1 < p.group) p.lse[head0 + n1] = lse1;
       }
     }
   }
   __syncthreads();
 }
 
-// One warp per (request, query head).
+// One CTA of 8 warps per (request, query head): merges the request's ranges.
+// All threads find the max and the sum of exp over the range LSEs; warp w
+// then accumulates ranges w, w+8, ... (four loads in flight per lane) and the
+// eight partial vectors are added in shared memory.  A request with one range
+// was written by the split kernel already; one with none (empty context)
+// gets O = 0 and LSE = -inf.
+constexpr int COMBINE_WARPS = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(COMBINE_WARPS * 32)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                   __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int rows, int S) {
-  const int r = blockIdx.x * 4 + warp_id();
-  const int lane = lane_id();
-  if (r >= rows) return;
+                   const int32_t* __restrict__ prefix, __nv_bfloat16* __restrict__ o,
+                   float* __restrict__ lse, int Hq, int S) {
+  constexpr int PER = D / 32;  // output elements per lane
+  __shared__ float red[COMBINE_WARPS][D];
+  __shared__ float wred[COMBINE_WARPS];
+  const int r = blockIdx.x;
+  const int b = r / Hq;
+  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  const int n = __ldg(prefix + b + 1) - __ldg(prefix + b);
+  if (n == 1) return;
   const float* lp = lse_part + (size_t)r * S;
   const float log2e = 1.4426950408889634f;
+  // max of the range LSEs
   float mx = -INFINITY;
-  for (int s = lane; s < S; s += 32) mx = fmaxf(mx, lp[s]);
+  for (int s = tid; s < n; s += COMBINE_WARPS * 32) mx = fmaxf(mx, lp[s]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  constexpr int PER = D / 32;
+  if (lane == 0) wred[warp] = mx;
+  __syncthreads();
+  mx = wred[0];
+#pragma unroll
+  for (int w = 1; w < COMBINE_WARPS; ++w) mx = fmaxf(mx, wred[w]);
+  __syncthreads();
+  float total_lse = -INFINITY;
   float out[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) out[i] = 0.f;
-  float total_lse = -INFINITY;
   if (mx != -INFINITY) {
     float sum = 0.f;
-    for (int s = lane; s < S; s += 32) sum += ex2((lp[s] - mx) * log2e);
+    for (int s = tid; s < n; s += COMBINE_WARPS * 32) sum += ex2((lp[s] - mx) * log2e);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) wred[warp] = sum;
+    __syncthreads();
+    sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < COMBINE_WARPS; ++w) sum += wred[w];
     total_lse = mx + __logf(sum);
     const float* op = o_part + (size_t)r * S * D + lane * PER;
-    for (int s = 0; s < S; ++s) {
-      const float w = ex2((lp[s] - total_lse) * log2e);
-      if (w == 0.f) continue;  // empty split (lse = -inf) or negligible
-      if constexpr (PER == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(op + (size_t)s * D);
-        out[0] += w * v.x;
-        out[1] += w * v.y;
-        out[2] += w * v.z;
-        out[3] += w * v.w;
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(op + (size_t)s * D);
-        out[0] += w * v.x;
-        out[1] += w * v.y;
+    int s = warp;
+    for (; s + 3 * COMBINE_WARPS < n; s += 4 * COMBINE_WARPS) {
+      float v[4][PER], w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int su = s + u * COMBINE_WARPS;
+        w[u] = ex2((lp[su] - total_lse) * log2e);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) v[u][i] = op[(size_t)su * D + i];
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < PER; ++i) out[i] = fmaf(w[u], v[u][i], out[i]);
+    }
+    for (; s < n; s += COMBINE_WARPS) {
+      const float w = ex2((lp[s] - total_lse) * log2e);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) out[i] = fmaf(w, op[(size_t)s * D + i], out[i]);
     }
   }
-  __nv_bfloat16* dst = o + (size_t)r * D + lane * PER;
 #pragma unroll
-  for (int i = 0; i < PER; i += 2)
-    *reinterpret_cast<uint32_t*>(dst + i) = pack_bf16x2(out[i], out[i + 1]);
-  if (lse && lane == 0) lse[r] = total_lse;
+  for (int i = 0; i < PER; ++i) red[warp][lane * PER + i] = out[i];
+  __syncthreads();
+  if (warp == 0) {
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      acc[i] = 0.f;
+#pragma unroll
+      for (int w = 0; w < COMBINE_WARPS; ++w) acc[i] += red[w][lane * PER + i];
+    }
+    __nv_bfloat16* dst = o + (size_t)r * D + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; i += 2)
+      *reinterpret_cast<uint32_t*>(dst + i) = pack_bf16x2(acc[i], acc[i + 1]);
+    if (lse && lane == 0) lse[r] = total_lse;
+  }
 }
 
 }  // namespace decode

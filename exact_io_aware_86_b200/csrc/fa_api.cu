@@ -139,13 +139,34 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Automatic page ranges for the decode: every range spans the same number of
+// pages, sized so the flat list of (range, kv-head group) items gives each
+// SM about eight of them (counting every request at max_blocks pages), and
+// never shorter than 512 tokens (so the per-range partial output stays a
+// small fraction of the bytes the range reads).
+int auto_chunk_pages(int B, int Hkv, int max_blocks, int page_size, int num_sms) {
+  const long long ngroups = Hkv / heads_per_cta(Hkv);
+  const long long upper = (long long)B * max_blocks * ngroups;
+  const long long target = 8LL * (num_sms > 0 ? num_sms : 148);
+  long long c = (upper + target - 1) / target;
+  const long long min_c = (512 + page_size - 1) / page_size;
+  if (c < min_c) c = min_c;
+  if (c > max_blocks) c = max_blocks;
+  if (c < 1) c = 1;
+  return (int)c;
+}
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
 template <int D>
 fa_status launch_decode(const void* q, const void* kp, const void* vp, const int32_t* bt,
-                        const int32_t* sl, int page_size, int S, void* o, cudaStream_t stream,
-                        int B, int Hq, int Hkv, int max_blocks, int num_pages, float scale,
-                        float* lse, void* ws) {
+                        const int32_t* sl, int page_size, int num_splits, void* o,
+                        cudaStream_t stream, int B, int Hq, int Hkv, int max_blocks, int num_pages,
+                        float scale, float* lse, void* ws) {
   using namespace fa::decode;
   const int hpb = heads_per_cta(Hkv);
+  const int sms = num_sms_current();
+  if (sms <= 0) return FA_ERR_CUDA;
   CUtensorMap tk, tv;
   {
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv,
@@ -164,27 +185,44 @@ fa_status launch_decode(const void* q, const void* kp, const void* vp, const int
   p.Hkv = Hkv;
   p.group = Hq / Hkv;
   p.hpb = hpb;
+  p.ngroups = Hkv / hpb;
   p.page_size = page_size;
   p.max_blocks = max_blocks;
   p.num_pages = num_pages;
-  p.num_splits = S;
+  if (num_splits == 0) {
+    p.chunk_pages = auto_chunk_pages(B, Hkv, max_blocks, page_size, sms);
+    p.s_max = ceil_div(max_blocks, p.chunk_pages);
+  } else {
+    p.chunk_pages = 0;
+    p.s_max = num_splits;
+  }
   p.half_bytes = Cfg<D>::PANELS * hpb * BOX_BYTES;
   p.scale_log2 = resolve_scale(scale, D) * kLog2e;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
-  const size_t opart_bytes = round_up((size_t)B * Hq * S * D * sizeof(float), 256);
-  p.o_part = S > 1 ? static_cast<float*>(ws) : nullptr;
-  p.lse_part = S > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + opart_bytes) : nullptr;
+  const bool split = p.s_max > 1;
+  const size_t opart_bytes = round_up((size_t)B * Hq * p.s_max * D * sizeof(float), 256);
+  const size_t lpart_bytes = round_up((size_t)B * Hq * p.s_max * sizeof(float), 256);
+  p.o_part = split ? static_cast<float*>(ws) : nullptr;
+  p.lse_part = split ? reinterpret_cast<float*>(static_cast<char*>(ws) + opart_bytes) : nullptr;
+  int32_t* prefix = split ? reinterpret_cast<int32_t*>(static_cast<char*>(ws) + opart_bytes + lpart_bytes)
+                          : nullptr;
+  p.split_prefix = prefix;
 
+  if (split) {
+    plan_kernel<<<1, 1024, 0, stream>>>(p, prefix);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
   const int smem = STAGES * stage_bytes(p.half_bytes) + 1024 + 64;
   static bool attr_ok = set_smem(split_kernel<D>, STAGES * stage_bytes(Cfg<D>::PANELS * MAX_HPB * BOX_BYTES) + 1024 + 64);
   if (!attr_ok) return FA_ERR_CUDA;
-  const dim3 grid((unsigned)S, (unsigned)(Hkv / hpb), (unsigned)B);
+  const long long upper = (split ? (long long)B * p.s_max : (long long)B) * p.ngroups;
+  const int grid = (int)(upper < sms ? upper : sms);
   split_kernel<D><<<grid, (hpb + 1) * 32, smem, stream>>>(tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  if (S > 1) {
-    const int rows = B * Hq;
-    combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(p.o_part, p.lse_part, p.o, lse, rows, S);
+  if (split) {
+    combine_kernel<D><<<B * Hq, COMBINE_WARPS * 32, 0, stream>>>(p.o_part, p.lse_part, prefix,
+                                                                 p.o, lse, Hq, p.s_max);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
@@ -221,20 +259,16 @@ size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits) {
   if (B <= 0 || Hq <= 0 || d <= 0 || num_splits <= 1) return 0;
   const size_t o_part = round_up((size_t)B * Hq * num_splits * d * sizeof(float), 256);
   const size_t l_part = round_up((size_t)B * Hq * num_splits * sizeof(float), 256);
-  return o_part + l_part;
+  const size_t prefix = round_up((size_t)(B + 1) * sizeof(int32_t), 256);
+  return o_part + l_part + prefix;
 }
 
-int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int num_sms) {
-  if (B <= 0 || Hkv <= 0 || max_blocks_per_seq <= 0) return 1;
+int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int page_size, int num_sms) {
+  if (B <= 0 || Hkv <= 0 || max_blocks_per_seq <= 0 || page_size <= 0) return 1;
   if (num_sms <= 0) num_sms = num_sms_current();
   if (num_sms <= 0) num_sms = 148;
-  const long long units = (long long)B * (Hkv / heads_per_cta(Hkv));
-  const long long target = 4LL * num_sms;  // work units to spread over the SMs
-  long long s = (target + units - 1) / units;
-  if (s > max_blocks_per_seq) s = max_blocks_per_seq;
-  if (s > 1024) s = 1024;
-  if (s < 1) s = 1;
-  return (int)s;
+  const int c = auto_chunk_pages(B, Hkv, max_blocks_per_seq, page_size, num_sms);
+  return ceil_div(max_blocks_per_seq, c);
 }
 
 fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
@@ -258,7 +292,8 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
     return FA_ERR_UNSUPPORTED;
   if (B > 65535 || Hkv / heads_per_cta(Hkv) > 65535) return FA_ERR_UNSUPPORTED;
   if (B == 0) return FA_OK;
-  const int S = num_splits == 0 ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, 0) : num_splits;
+  const int S = num_splits == 0 ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, page_size, 0)
+                                : num_splits;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t need = fa_decode_workspace_size(B, Hq, d, S);
   void* ws = workspace;
@@ -273,11 +308,11 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
   }
   fa_status st;
   if (d == 64)
-    st = launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, page_size, S, o, s, B, Hq,
-                           Hkv, max_blocks_per_seq, num_pages, scale, lse, ws);
+    st = launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, page_size, num_splits, o, s,
+                           B, Hq, Hkv, max_blocks_per_seq, num_pages, scale, lse, ws);
   else
-    st = launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, page_size, S, o, s, B,
-                            Hq, Hkv, max_blocks_per_seq, num_pages, scale, lse, ws);
+    st = launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, page_size, num_splits, o,
+                            s, B, Hq, Hkv, max_blocks_per_seq, num_pages, scale, lse, ws);
   if (owned && cudaFreeAsync(ws, s) != cudaSuccess && st == FA_OK) st = FA_ERR_CUDA;
   return st;
 }
@@ -360,7 +395,7 @@ int fa_version(void) { return 100; }
 // --------------------------------------------------------------------------
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per device
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
@@ -392,7 +427,9 @@ extern "C" fa_status fa_decode_paged_noalloc(const void* q, const void* k_pages,
                                              int Hq, int Hkv, int d, int max_blocks_per_seq,
                                              int num_pages, float scale, float* lse) {
   if (num_splits < 0 || B < 0 || Hq <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
-  const int S = num_splits == 0 ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, 0) : num_splits;
+  const int S = num_splits == 0
+                    ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, page_size, 0)
+                    : num_splits;
   const size_t need = fa_decode_workspace_size(B, Hq, d, S);
   if (need > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
@@ -400,7 +437,8 @@ extern "C" fa_status fa_decode_paged_noalloc(const void* q, const void* k_pages,
     scratch = decode_scratch_on_current_device();
     if (!scratch) return FA_ERR_CUDA;
   }
-  return fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, page_size, S, o, stream, B,
-                         Hq, Hkv, d, max_blocks_per_seq, num_pages, scale, lse, scratch,
+  // num_splits is passed on unchanged, so 0 keeps the automatic page ranges
+  return fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, page_size, num_splits, o,
+                         stream, B, Hq, Hkv, d, max_blocks_per_seq, num_pages, scale, lse, scratch,
                          need > 0 ? kNoAllocScratchBytes : 0);
 }

@@ -93,10 +93,11 @@ fa_status fa_prefill(const void *q, const void *k, const void *v, void *o, float
  *   seq_lens     int32 [B]  device; context length of each request,
  *                0 <= seq_lens[b] <= max_blocks_per_seq * page_size
  *   page_size    tokens per page (>= 1)
- *   num_splits   number of contiguous page ranges each request's context is
- *                cut into (0 = choose automatically, see
- *                fa_decode_auto_splits); the result does not depend on it
- *                beyond rounding
+ *   num_splits   number of contiguous, near-equal page ranges each
+ *                request's context is cut into; 0 = automatic: ranges of one
+ *                fixed page count for all requests (see
+ *                fa_decode_auto_splits).  The result does not depend on the
+ *                partition beyond rounding.
  *   o            bf16 [B, Hq, d]  output (written)
  *   lse          fp32 [B, Hq]  natural-log log-sum-exp, or NULL
  *   workspace    device scratch of at least
@@ -115,7 +116,7 @@ fa_status fa_decode_paged(const void *q, const void *k_pages, const void *v_page
 /*
  * Paged decode that allocates nothing (no counterpart in the pages; this is
  * a deployment convenience).  Same arguments and result as fa_decode_paged
- * without the workspace pair: the split scratch comes from a 16 MiB array
+ * without the workspace pair: the split scratch comes from a 64 MiB array
  * compiled into the library, held by every GPU that loads it until exit.
  *
  * For callers that cannot allocate device memory when they run a decode
@@ -125,7 +126,7 @@ fa_status fa_decode_paged(const void *q, const void *k_pages, const void *v_page
  *
  *   - Returns FA_ERR_UNSUPPORTED, launching nothing, when
  *     fa_decode_workspace_size(B, Hq, d, resolved num_splits) exceeds
- *     16 MiB; use fewer splits or fa_decode_paged with your own workspace.
+ *     64 MiB; use fewer splits or fa_decode_paged with your own workspace.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make
  *     that first call before any stream capture.
@@ -140,13 +141,17 @@ fa_status fa_decode_paged_noalloc(const void *q, const void *k_pages, const void
                                   int num_pages, float scale, float *lse);
 
 /* Bytes of workspace fa_decode_paged needs for this shape and split count
- * (partial outputs fp32 [B, Hq, S, d] and partial LSEs fp32 [B, Hq, S]). */
+ * (partial outputs fp32 [B, Hq, S, d], partial LSEs fp32 [B, Hq, S] and
+ * the per-request range counts int32 [B+1]); 0 when S <= 1. */
 size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits);
 
-/* The split count num_splits = 0 resolves to: enough (request, split) work
- * units to give every SM several to run, and no more splits than the
- * longest context has pages.  num_sms <= 0 queries the current device. */
-int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int num_sms);
+/* The split count num_splits = 0 resolves to.  In that automatic mode every
+ * page range spans the same number of pages c (about eight ranges per SM,
+ * counting every request at max_blocks_per_seq pages, and at least 512
+ * tokens), and this returns ceil(max_blocks_per_seq / c): the largest number
+ * of ranges any request can have, which sizes the workspace.  num_sms <= 0
+ * queries the current device. */
+int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int page_size, int num_sms);
 
 /*
  * fp32 debug paths: the same operations with fp32 q/k/v/o (layouts as

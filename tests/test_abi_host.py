@@ -99,22 +99,28 @@ def test_decode_argument_checks(lib):
 
 
 def test_decode_workspace_is_linear_in_splits_not_context(lib):
-    """The split workspace holds fp32 partial outputs and LSEs:
-    B*Hq*S*(d+1) floats (rounded to 256-byte blocks), independent of the
-    context length -- nothing of size N^2 (or even N) is ever allocated."""
-    for B, Hq, d, S in ((64, 32, 128, 10), (2, 32, 128, 296), (1, 1, 64, 2)):
+    """The split workspace holds fp32 partial outputs and LSEs,
+    B*Hq*S*(d+1) floats, plus B+1 range counts (each part rounded to
+    256-byte blocks), independent of the context length -- nothing of size
+    N^2 (or even N) is ever allocated."""
+    for B, Hq, d, S in ((64, 32, 128, 19), (2, 32, 128, 256), (1, 1, 64, 2)):
         n = lib.fa_decode_workspace_size(B, Hq, d, S)
-        assert n >= B * Hq * S * (d + 1) * 4
-        assert n <= B * Hq * S * (d + 1) * 4 + 512
+        assert n >= B * Hq * S * (d + 1) * 4 + (B + 1) * 4
+        assert n <= B * Hq * S * (d + 1) * 4 + (B + 1) * 4 + 768
     assert lib.fa_decode_workspace_size(64, 32, 128, 1) == 0
 
 
 def test_auto_splits_rule(lib):
-    # enough (request, split) units for several per SM, capped by the page count
-    assert lib.fa_decode_auto_splits(64, 8, 2048, 148) == 10
-    assert lib.fa_decode_auto_splits(2, 8, 2048, 148) == 296
-    assert lib.fa_decode_auto_splits(2, 8, 3, 148) == 3
-    assert lib.fa_decode_auto_splits(10000, 8, 64, 148) == 1
+    """Automatic ranges span c pages: about 8 ranges per SM counting every
+    request at max_blocks pages, at least 512 tokens, at most max_blocks;
+    the call returns ceil(max_blocks / c)."""
+    # 64 requests x 2048 pages of 16 tokens: c = ceil(131072 / 1184) = 111
+    assert lib.fa_decode_auto_splits(64, 8, 2048, 16, 148) == 19
+    # 2 requests x 2048 pages of 64 tokens: 4 pages would be < 512 tokens -> c = 8
+    assert lib.fa_decode_auto_splits(2, 8, 2048, 64, 148) == 256
+    # short contexts: one range per request
+    assert lib.fa_decode_auto_splits(2, 8, 3, 16, 148) == 1
+    assert lib.fa_decode_auto_splits(10000, 8, 64, 16, 148) == 1
 
 
 def test_python_binding_rejects_host_tensors():

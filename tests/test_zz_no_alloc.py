@@ -43,8 +43,8 @@ def test_noalloc_rejects_scratch_beyond_its_maximum():
     q, kp, vp, bt, sl = (t.cuda() for t in (inp.q, inp.k_pages, inp.v_pages, inp.block_table,
                                              inp.seq_lens))
     o = torch.empty_like(q)
-    splits = 1024  # 4 * 32 * 1024 * 129 * 4 bytes > 16 MiB
-    assert api.decode_workspace_size(4, 32, 128, splits) > 16 << 20
+    splits = 2048  # 4 * 32 * 2048 * 129 * 4 bytes > 64 MiB
+    assert api.decode_workspace_size(4, 32, 128, splits) > 64 << 20
     with pytest.raises(api.FAError) as e:
         api.fa_decode_paged_noalloc(q, kp, vp, bt, sl, splits, o)
     assert e.value.code == api.FA_ERR_UNSUPPORTED
