@@ -298,8 +298,8 @@ class DeviceWorkload:
             self.bt, self.sl = din.block_table.to(dev), din.seq_lens.to(dev)
             # automatic page ranges (num_splits = 0); splits = the most ranges a
             # request can get, which sizes the workspace
-            self.splits = api.decode_auto_splits(din.B, din.Hkv, din.block_table.shape[1],
-                                                 din.page_size)
+            self.splits = api.decode_auto_splits(din.B, din.Hq, din.Hkv,
+                                                 din.block_table.shape[1], din.page_size)
             nbytes = api.decode_workspace_size(din.B, din.Hq, din.d, self.splits)
             self.ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) if nbytes else None
             self.do = torch.empty_like(self.dq)

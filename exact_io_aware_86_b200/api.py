@@ -50,7 +50,7 @@ def load_library(path: str = LIB_PATH):
     lib.fa_decode_paged_noalloc.restype = ctypes.c_int
     lib.fa_decode_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.fa_decode_workspace_size.restype = sz
-    lib.fa_decode_auto_splits.argtypes = [i32, i32, i32, i32, i32]
+    lib.fa_decode_auto_splits.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.fa_prefill_f32.argtypes = lib.fa_prefill.argtypes
     lib.fa_decode_paged_f32.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
                                         i32, f32, vp]
@@ -154,10 +154,10 @@ def decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:
     return int(load_library().fa_decode_workspace_size(B, Hq, d, num_splits))
 
 
-def decode_auto_splits(B: int, Hkv: int, max_blocks_per_seq: int, page_size: int,
+def decode_auto_splits(B: int, Hq: int, Hkv: int, max_blocks_per_seq: int, page_size: int,
                        num_sms: int = 0) -> int:
     """The split count ``num_splits = 0`` resolves to (sizes the workspace)."""
-    return int(load_library().fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, page_size,
+    return int(load_library().fa_decode_auto_splits(B, Hq, Hkv, max_blocks_per_seq, page_size,
                                                     num_sms))
 
 
@@ -228,7 +228,7 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int = 0
     ``fa_decode_paged``.  Returns (o, lse or None)."""
     B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
         q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16)
-    S = num_splits if num_splits > 0 else decode_auto_splits(B, Hkv, max_blocks, page_size)
+    S = num_splits if num_splits > 0 else decode_auto_splits(B, Hq, Hkv, max_blocks, page_size)
     o = torch.empty_like(q)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if return_lse else None
     nbytes = decode_workspace_size(B, Hq, d, S)

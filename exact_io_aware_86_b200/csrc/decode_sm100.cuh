@@ -19,8 +19,8 @@
 //   c + #CTAs, ... of the flat list (each for a group of up to 8 kv heads).
 //   A producer warp gathers each range's pages 16 tokens at a time
 //   into a shared-memory ring with TMA (3-D tensor maps over the pool with
-//   128-byte swizzle, one 16-token box per kv head and 64-wide half of
-//   head_dim; page_size is a multiple of 16).  Each consumer warp owns one kv head and the Hq/Hkv <= 8 query
+//   128-byte swizzle, one 16-token box of all the CTA's kv heads per 64-wide
+//   half of head_dim; page_size is a multiple of 16).  Each consumer warp owns one kv head and the Hq/Hkv <= 8 query
 //   heads that read it, so every K/V byte is read from HBM once for the whole
 //   group.  Scores and the P V product use warp-level bf16 tensor-core MMAs
 //   (S^T = K Q^T with tokens as rows, O^T += V^T P^T); the online softmax
@@ -68,11 +68,17 @@ struct Cfg {
   static constexpr int KS = D / 16;  // MMA k-steps over head_dim / m-tiles over head_dim
 };
 
-// One TMA box = 16 tokens x 64 head_dim elements of one kv head (2 KB), 128 B
-// per row.  Shared-memory layout of the K (or V) half of a stage:
-// [panel][kv head][token][128 B]; every box starts on a 1024-byte boundary
-// and the TMA 128-byte swizzle XORs the 16-byte chunk index with (token & 7).
-constexpr int BOX_BYTES = TOK * 128;
+// The pool is seen by TMA as a 3-D tensor with dimensions ordered (head_dim,
+// token, kv head) -- strides 2*Hkv*D and 2*D bytes -- so one box {64 dims,
+// 16 tokens, hpb heads} lands in shared memory as [kv head][token][128 B].
+// Layout of the K (or V) half of a stage: [panel][kv head][token][128 B];
+// each panel's box starts on a 1024-byte boundary and the 128-byte swizzle
+// XORs the 16-byte chunk index with (token & 7), so the eight token rows an
+// ldmatrix reads for one head fall in different banks.  Two boxes per
+// stage for K and two for V (d = 128): few, large TMA operations -- with a
+// box per head the gather ran at ~70% of HBM bandwidth, with one box for all
+// heads at ~98%.
+constexpr int BOX_BYTES = TOK * 128;  // one head's 16 token rows of one panel
 
 __host__ __device__ inline int stage_bytes(int half_bytes) { return 2 * half_bytes; }
 
@@ -243,12 +249,12 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
           mbar_arrive_expect_tx(&full[slot], 2 * p.half_bytes);
           uint8_t* kdst = smem + slot * sbytes;
           uint8_t* vdst = kdst + p.half_bytes;
-          for (int pn = 0; pn < C::PANELS; ++pn)
-            for (int hh = 0; hh < p.hpb; ++hh) {
-              const int off = (pn * p.hpb + hh) * BOX_BYTES;
-              tma_load_3d(kdst + off, &tmK, &full[slot], pn * 64, kvh0 + hh, z);
-              tma_load_3d(vdst + off, &tmV, &full[slot], pn * 64, kvh0 + hh, z);
-            }
+          // one box per 64-wide half of head_dim holds all the CTA's kv heads
+          for (int pn = 0; pn < C::PANELS; ++pn) {
+            const int off = pn * p.hpb * BOX_BYTES;
+            tma_load_3d(kdst + off, &tmK, &full[slot], pn * 64, z, kvh0);
+            tma_load_3d(vdst + off, &tmV, &full[slot], pn * 64, z, kvh0);
+          }
         }
       }
       // every load issued must land before the CTA exits

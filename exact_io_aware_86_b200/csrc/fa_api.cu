@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -139,24 +140,48 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
 // Automatic page ranges for the decode: every range spans the same number of
-// pages, sized so the flat list of (range, kv-head group) items gives each
-// SM about eight of them (counting every request at max_blocks pages), and
-// never shorter than 512 tokens (so the per-range partial output stays a
-// small fraction of the bytes the range reads).
-int auto_chunk_pages(int B, int Hkv, int max_blocks, int page_size, int num_sms) {
-  const long long ngroups = Hkv / heads_per_cta(Hkv);
-  const long long upper = (long long)B * max_blocks * ngroups;
-  const long long target = 8LL * (num_sms > 0 ? num_sms : 148);
-  long long c = (upper + target - 1) / target;
-  const long long min_c = (512 + page_size - 1) / page_size;
-  if (c < min_c) c = min_c;
-  if (c > max_blocks) c = max_blocks;
-  if (c < 1) c = 1;
-  return (int)c;
+// pages c.  The range count is planned as if every request had max_blocks
+// pages; c is picked among the sizes that give r = 1..32 rounds of ranges
+// per SM, maximising a simple model: (load balance of the last round) x
+// (1 - the partial-output traffic relative to the K/V bytes - a fixed
+// per-range cost), with ranges of at least 256 tokens.
+int auto_chunk_pages(int B, int Hq, int Hkv, int max_blocks, int page_size, int num_sms) {
+  const int hpb = heads_per_cta(Hkv);
+  const long long ngroups = Hkv / hpb;
+  const int G = num_sms > 0 ? num_sms : 148;
+  const long long U = (long long)B * max_blocks * ngroups;
+  const int c_min = std::min(max_blocks, std::max(1, ceil_div(256, page_size)));
+  const double qpk = (double)Hq / Hkv;
+  auto score = [&](int c) {
+    const long long ranges = ceil_div(max_blocks, c);
+    const long long items = (long long)B * ranges * ngroups;
+    const double rounds = (double)items / G;
+    const double bal = items >= G ? rounds / std::ceil(rounds) : rounds;
+    // fp32 partial O and LSE, written and read once, per byte of K and V
+    const double part = ranges > 1 ? 2.0 * qpk / ((double)c * page_size) : 0.0;
+    // about 0.5 us of per-range work at ~40 GB/s per SM, per byte a range reads
+    const double fixed = 20000.0 / ((double)c * page_size * hpb * 512.0);
+    return bal * (1.0 - part - fixed);
+  };
+  int best_c = max_blocks;
+  double best = score(max_blocks);
+  for (int r = 1; r <= 32; ++r) {
+    long long c = (U + (long long)r * G - 1) / ((long long)r * G);
+    for (long long cc = c - 1; cc <= c + 1; ++cc) {
+      const int ci = (int)std::max<long long>(c_min, std::min<long long>(cc, max_blocks));
+      const double sc = score(ci);
+      if (sc > best + 1e-9) {
+        best = sc;
+        best_c = ci;
+      }
+    }
+  }
+  return best_c;
 }
 
-int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 template <int D>
 fa_status launch_decode(const void* q, const void* kp, const void* vp, const int32_t* bt,
@@ -169,10 +194,12 @@ fa_status launch_decode(const void* q, const void* kp, const void* vp, const int
   if (sms <= 0) return FA_ERR_CUDA;
   CUtensorMap tk, tv;
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv,
-                                (cuuint64_t)num_pages * (cuuint64_t)page_size};
-    const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)TOK};
+    // dimensions (head_dim, token, kv head): a box of the CTA's heads lands in
+    // shared memory as [head][token][64 dims] (see decode_sm100.cuh)
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)num_pages * (cuuint64_t)page_size,
+                                (cuuint64_t)Hkv};
+    const cuuint64_t str[2] = {(cuuint64_t)Hkv * D * 2, (cuuint64_t)D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)TOK, (cuuint32_t)hpb};
     if (!make_map(&tk, kp, 3, dims, str, box)) return FA_ERR_CUDA;
     if (!make_map(&tv, vp, 3, dims, str, box)) return FA_ERR_CUDA;
   }
@@ -190,7 +217,7 @@ fa_status launch_decode(const void* q, const void* kp, const void* vp, const int
   p.max_blocks = max_blocks;
   p.num_pages = num_pages;
   if (num_splits == 0) {
-    p.chunk_pages = auto_chunk_pages(B, Hkv, max_blocks, page_size, sms);
+    p.chunk_pages = auto_chunk_pages(B, Hq, Hkv, max_blocks, page_size, sms);
     p.s_max = ceil_div(max_blocks, p.chunk_pages);
   } else {
     p.chunk_pages = 0;
@@ -263,11 +290,14 @@ size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits) {
   return o_part + l_part + prefix;
 }
 
-int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int page_size, int num_sms) {
-  if (B <= 0 || Hkv <= 0 || max_blocks_per_seq <= 0 || page_size <= 0) return 1;
+int fa_decode_auto_splits(int B, int Hq, int Hkv, int max_blocks_per_seq, int page_size,
+                          int num_sms) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_blocks_per_seq <= 0 ||
+      page_size <= 0)
+    return 1;
   if (num_sms <= 0) num_sms = num_sms_current();
   if (num_sms <= 0) num_sms = 148;
-  const int c = auto_chunk_pages(B, Hkv, max_blocks_per_seq, page_size, num_sms);
+  const int c = auto_chunk_pages(B, Hq, Hkv, max_blocks_per_seq, page_size, num_sms);
   return ceil_div(max_blocks_per_seq, c);
 }
 
@@ -292,8 +322,9 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
     return FA_ERR_UNSUPPORTED;
   if (B > 65535 || Hkv / heads_per_cta(Hkv) > 65535) return FA_ERR_UNSUPPORTED;
   if (B == 0) return FA_OK;
-  const int S = num_splits == 0 ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, page_size, 0)
-                                : num_splits;
+  const int S = num_splits == 0
+                    ? fa_decode_auto_splits(B, Hq, Hkv, max_blocks_per_seq, page_size, 0)
+                    : num_splits;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t need = fa_decode_workspace_size(B, Hq, d, S);
   void* ws = workspace;
@@ -428,7 +459,7 @@ extern "C" fa_status fa_decode_paged_noalloc(const void* q, const void* k_pages,
                                              int num_pages, float scale, float* lse) {
   if (num_splits < 0 || B < 0 || Hq <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
   const int S = num_splits == 0
-                    ? fa_decode_auto_splits(B, Hkv, max_blocks_per_seq, page_size, 0)
+                    ? fa_decode_auto_splits(B, Hq, Hkv, max_blocks_per_seq, page_size, 0)
                     : num_splits;
   const size_t need = fa_decode_workspace_size(B, Hq, d, S);
   if (need > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;

@@ -146,12 +146,13 @@ fa_status fa_decode_paged_noalloc(const void *q, const void *k_pages, const void
 size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits);
 
 /* The split count num_splits = 0 resolves to.  In that automatic mode every
- * page range spans the same number of pages c (about eight ranges per SM,
- * counting every request at max_blocks_per_seq pages, and at least 512
- * tokens), and this returns ceil(max_blocks_per_seq / c): the largest number
- * of ranges any request can have, which sizes the workspace.  num_sms <= 0
- * queries the current device. */
-int fa_decode_auto_splits(int B, int Hkv, int max_blocks_per_seq, int page_size, int num_sms);
+ * page range spans the same number of pages c, chosen for whole rounds of
+ * ranges per SM (counting every request at max_blocks_per_seq pages) with
+ * little partial-output traffic, and at least 256 tokens; this returns
+ * ceil(max_blocks_per_seq / c): the largest number of ranges any request can
+ * have, which sizes the workspace.  num_sms <= 0 queries the current device. */
+int fa_decode_auto_splits(int B, int Hq, int Hkv, int max_blocks_per_seq, int page_size,
+                          int num_sms);
 
 /*
  * fp32 debug paths: the same operations with fp32 q/k/v/o (layouts as

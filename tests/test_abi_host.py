@@ -111,16 +111,19 @@ def test_decode_workspace_is_linear_in_splits_not_context(lib):
 
 
 def test_auto_splits_rule(lib):
-    """Automatic ranges span c pages: about 8 ranges per SM counting every
-    request at max_blocks pages, at least 512 tokens, at most max_blocks;
-    the call returns ceil(max_blocks / c)."""
-    # 64 requests x 2048 pages of 16 tokens: c = ceil(131072 / 1184) = 111
-    assert lib.fa_decode_auto_splits(64, 8, 2048, 16, 148) == 19
-    # 2 requests x 2048 pages of 64 tokens: 4 pages would be < 512 tokens -> c = 8
-    assert lib.fa_decode_auto_splits(2, 8, 2048, 64, 148) == 256
-    # short contexts: one range per request
-    assert lib.fa_decode_auto_splits(2, 8, 3, 16, 148) == 1
-    assert lib.fa_decode_auto_splits(10000, 8, 64, 16, 148) == 1
+    """Automatic ranges span c pages, chosen for whole rounds of ranges per
+    SM with little partial-output traffic (at least 256 tokens, at most
+    max_blocks); the call returns ceil(max_blocks / c)."""
+    # 64 requests x 2048 pages of 16 tokens: c = 69 pages, 30 ranges at most,
+    # 64 * 30 = 1920 ranges = 12.97 rounds of 148
+    assert lib.fa_decode_auto_splits(64, 32, 8, 2048, 16, 148) == 30
+    # 2 requests x 2048 pages of 64 tokens: c = 28, 2 * 74 = 148 ranges, one round
+    assert lib.fa_decode_auto_splits(2, 32, 8, 2048, 64, 148) == 74
+    # short contexts or many requests: one range per request
+    assert lib.fa_decode_auto_splits(2, 32, 8, 3, 16, 148) == 1
+    assert lib.fa_decode_auto_splits(10000, 32, 8, 64, 16, 148) == 1
+    # invalid shapes fall back to one range
+    assert lib.fa_decode_auto_splits(2, 12, 8, 64, 16, 148) == 1
 
 
 def test_python_binding_rejects_host_tensors():
