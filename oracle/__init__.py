@@ -63,6 +63,26 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _ptr_or_null(a):
+    return None if a is None else _ptr(a)
+
+
+def _variant(window, softcap, alibi_slopes, B: int, Hq: int):
+    """Marshals the mask-variant arguments: (left, right, softcap, slopes
+    as contiguous float32 or None, slope stride per sequence)."""
+    left, right = (int(window[0]), int(window[1]))
+    if softcap < 0:
+        raise ValueError("softcap must be >= 0")
+    if alibi_slopes is None:
+        return left, right, float(softcap), None, 0
+    a = np.ascontiguousarray(_as_np(alibi_slopes)[0], dtype=np.float32)
+    if a.shape == (Hq,):
+        return left, right, float(softcap), a, 0
+    if a.shape == (B, Hq):
+        return left, right, float(softcap), a, Hq
+    raise ValueError(f"alibi_slopes must be [Hq] or [B, Hq], got {a.shape}")
+
+
 def _same_dtype(*arrs):
     codes = {c for _, c in arrs}
     if len(codes) != 1:
@@ -77,15 +97,17 @@ class Oracle:
         lib = ctypes.CDLL(path)
         vp = ctypes.c_void_p
         ci, cd, c64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
-        lib.oracle_prefill_rows.argtypes = [vp, vp, vp, ci, vp, ci, ci, ci, ci, ci, cd,
-                                            vp, vp, c64, vp, vp]
-        lib.oracle_prefill.argtypes = [vp, vp, vp, ci, vp, ci, ci, ci, ci, ci, cd, vp, vp]
-        lib.oracle_prefill_probs.argtypes = [vp, vp, ci, vp, ci, ci, ci, ci, ci, cd, ci, ci, vp]
+        lib.oracle_prefill_rows_ex.argtypes = [vp, vp, vp, ci, vp, ci, ci, ci, ci, ci, cd,
+                                               ci, ci, cd, vp, ci, vp, vp, c64, vp, vp]
+        lib.oracle_prefill_ex.argtypes = [vp, vp, vp, ci, vp, ci, ci, ci, ci, ci, cd,
+                                          ci, ci, cd, vp, ci, vp, vp]
+        lib.oracle_prefill_probs.argtypes = [vp, vp, ci, vp, ci, ci, ci, ci, ci, cd,
+                                             ci, ci, cd, vp, ci, ci, ci, vp]
         lib.oracle_decode_paged.argtypes = [vp, vp, vp, ci, vp, vp, ci, ci, ci, ci, ci, ci,
                                             c64, cd, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_set_num_threads.argtypes = [ci]
-        for f in (lib.oracle_prefill_rows, lib.oracle_prefill, lib.oracle_prefill_probs,
+        for f in (lib.oracle_prefill_rows_ex, lib.oracle_prefill_ex, lib.oracle_prefill_probs,
                   lib.oracle_decode_paged, lib.oracle_num_threads):
             f.restype = ctypes.c_int
         lib.oracle_set_num_threads.restype = None
@@ -98,10 +120,15 @@ class Oracle:
     def num_threads(self) -> int:
         return int(self._lib.oracle_num_threads())
 
-    def prefill(self, q, k, v, cu_seqlens, causal: bool, scale: float):
+    def prefill(self, q, k, v, cu_seqlens, causal: bool, scale: float, window=(-1, -1),
+                softcap: float = 0.0, alibi_slopes=None):
         """Exact attention over packed sequences.
 
         q: [T, Hq, d]; k, v: [T, Hkv, d]; cu_seqlens: [B+1].
+        window = (left, right): key j visible to query i when
+        i - left <= j <= i + right (a negative bound: unlimited).
+        softcap > 0: logits x become softcap * tanh(x / softcap).
+        alibi_slopes: fp32 [Hq] or [B, Hq], adds -slope * |i - j|.
         Returns (o [T, Hq, d] float64, lse [Hq, T] float64).
         """
         (qa, c1), (ka, c2), (va, c3) = _as_np(q), _as_np(k), _as_np(v)
@@ -112,15 +139,19 @@ class Oracle:
         B = cu.shape[0] - 1
         o = np.zeros((T, Hq, d), np.float64)
         lse = np.zeros((Hq, T), np.float64)
-        rc = self._lib.oracle_prefill(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(cu), B, Hq, Hkv,
-                                      d, int(bool(causal)), float(scale), _ptr(o), _ptr(lse))
+        wl, wr, sc, al, ast = _variant(window, softcap, alibi_slopes, B, Hq)
+        rc = self._lib.oracle_prefill_ex(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(cu), B, Hq, Hkv,
+                                         d, int(bool(causal)), float(scale), wl, wr, sc,
+                                         _ptr_or_null(al), ast, _ptr(o), _ptr(lse))
         if rc != 0:
             raise ValueError(f"oracle_prefill rejected its arguments (rc={rc})")
         return o, lse
 
     def prefill_rows(self, q, k, v, cu_seqlens, causal: bool, scale: float,
-                     rows_t: Sequence[int], rows_h: Sequence[int]):
-        """Exact attention for selected (token, head) rows only.
+                     rows_t: Sequence[int], rows_h: Sequence[int], window=(-1, -1),
+                     softcap: float = 0.0, alibi_slopes=None):
+        """Exact attention for selected (token, head) rows only (variant
+        arguments as in ``prefill``).
 
         Returns (o [n, d] float64, lse [n] float64).  Rows are independent,
         so a sample of rows is exact for those rows.
@@ -136,16 +167,19 @@ class Oracle:
         n = rt.shape[0]
         o = np.zeros((n, d), np.float64)
         lse = np.zeros((n,), np.float64)
-        rc = self._lib.oracle_prefill_rows(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(cu), B, Hq,
-                                           Hkv, d, int(bool(causal)), float(scale), _ptr(rt),
-                                           _ptr(rh), n, _ptr(o), _ptr(lse))
+        wl, wr, sc, al, ast = _variant(window, softcap, alibi_slopes, B, Hq)
+        rc = self._lib.oracle_prefill_rows_ex(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(cu), B, Hq,
+                                              Hkv, d, int(bool(causal)), float(scale), wl, wr,
+                                              sc, _ptr_or_null(al), ast, _ptr(rt), _ptr(rh), n,
+                                              _ptr(o), _ptr(lse))
         if rc != 0:
             raise ValueError(f"oracle_prefill_rows rejected its arguments (rc={rc})")
         return o, lse
 
     def prefill_probs(self, q, k, cu_seqlens, causal: bool, scale: float, b: int, h: int,
-                      Hkv: int):
-        """The [L, L] probability matrix P of one (sequence, head); zeros where masked."""
+                      Hkv: int, window=(-1, -1), softcap: float = 0.0, alibi_slopes=None):
+        """The [L, L] probability matrix P of one (sequence, head); zeros where
+        masked (variant arguments as in ``prefill``)."""
         (qa, c1), (ka, c2) = _as_np(q), _as_np(k)
         dt = _same_dtype((qa, c1), (ka, c2))
         cu = _int_np(cu_seqlens, np.int32)
@@ -153,9 +187,10 @@ class Oracle:
         B = cu.shape[0] - 1
         L = int(cu[b + 1] - cu[b])
         P = np.zeros((L, L), np.float64)
+        wl, wr, sc, al, ast = _variant(window, softcap, alibi_slopes, B, Hq)
         rc = self._lib.oracle_prefill_probs(_ptr(qa), _ptr(ka), dt, _ptr(cu), B, Hq, Hkv, d,
-                                            int(bool(causal)), float(scale), int(b), int(h),
-                                            _ptr(P))
+                                            int(bool(causal)), float(scale), wl, wr, sc,
+                                            _ptr_or_null(al), ast, int(b), int(h), _ptr(P))
         if rc != 0:
             raise ValueError(f"oracle_prefill_probs rejected its arguments (rc={rc})")
         return P

@@ -26,6 +26,15 @@
  *  - The log-sum-exp of each row (natural log, of the scaled logits) is
  *    returned beside O; the pages name the row max m and sum l, and
  *    LSE = m + ln l.
+ *  - "flash-attention" skill page, section 3.3 (advanced features): a
+ *    sliding window window_size = (left, right) -- key j is visible to query
+ *    i when i - left <= j <= i + right, a negative bound meaning no limit on
+ *    that side ((4096, 0) looks 4096 tokens to the left); softcapping, which
+ *    replaces each logit x by softcap * tanh(x / softcap); and ALiBi slopes of
+ *    shape (nheads,) or (batch, nheads), read as the linear distance penalty
+ *    -slope * |i - j| added to the logit of query i and key j.  Logit here
+ *    means the scaled score scale * <q, k>; the cap is applied first and the
+ *    ALiBi penalty is added to the capped value.
  *
  * Precision: every product and sum is in double.  Inputs are read in the
  * caller's element type (bf16 bit patterns, fp32 or fp64) and upcast
@@ -61,16 +70,38 @@ static double elem(const void *base, size_t i, int dtype)
 }
 
 /*
+ * The logits of one query row against an explicit list of key rows:
+ * s_j = scale * <q, k_j>, then softcap * tanh(s_j / softcap) when
+ * softcap > 0, then + bias[j] when bias is not NULL.
+ */
+static void row_logits(const void *q, const void *k, int dtype, size_t qrow,
+                       const size_t *krows, size_t n, int d, double scale, double softcap,
+                       const double *bias, double *s)
+{
+    for (size_t j = 0; j < n; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c)
+            dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);
+        s[j] = scale * dot;
+        if (softcap > 0.0)
+            s[j] = softcap * tanh(s[j] / softcap);
+        if (bias)
+            s[j] += bias[j];
+    }
+}
+
+/*
  * One query row against an explicit list of key/value rows.
  *   qrow: element offset of the query vector (d consecutive elements)
  *   krows/vrows: element offsets of each visible key/value vector
  *   n: number of visible keys (n == 0 gives O = 0, LSE = -inf)
+ *   softcap, bias: logit modifiers of row_logits (0 / NULL for none)
  * s and p are caller scratch of length >= n.
  */
 static void attend_one_row(const void *q, const void *k, const void *v, int dtype,
                            size_t qrow, const size_t *krows, const size_t *vrows,
-                           size_t n, int d, double scale, double *s, double *p,
-                           double *o_out, double *lse_out)
+                           size_t n, int d, double scale, double softcap, const double *bias,
+                           double *s, double *p, double *o_out, double *lse_out)
 {
     if (n == 0) {
         for (int c = 0; c < d; ++c)
@@ -78,13 +109,7 @@ static void attend_one_row(const void *q, const void *k, const void *v, int dtyp
         *lse_out = -INFINITY;
         return;
     }
-    /* S_j = scale * <q, k_j> */
-    for (size_t j = 0; j < n; ++j) {
-        double dot = 0.0;
-        for (int c = 0; c < d; ++c)
-            dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);
-        s[j] = scale * dot;
-    }
+    row_logits(q, k, dtype, qrow, krows, n, d, scale, softcap, bias, s);
     /* softmax, pass 1: the row max */
     double m = s[0];
     for (size_t j = 1; j < n; ++j)
@@ -118,20 +143,50 @@ static int seq_of_token(const int32_t *cu, int B, int64_t t)
 }
 
 /*
+ * Whether key j is visible to query i, both local indices in a sequence of L
+ * tokens: j in [0, L); causal keeps j <= i; window_left >= 0 keeps
+ * j >= i - window_left; window_right >= 0 keeps j <= i + window_right.
+ */
+static int key_visible(int64_t i, int64_t j, int64_t L, int causal, int window_left,
+                       int window_right)
+{
+    if (j < 0 || j >= L)
+        return 0;
+    if (causal && j > i)
+        return 0;
+    if (window_left >= 0 && j < i - window_left)
+        return 0;
+    if (window_right >= 0 && j > i + window_right)
+        return 0;
+    return 1;
+}
+
+/* The ALiBi slope of (sequence b, query head h): alibi[b * stride + h]
+ * (stride 0 for one slope per head, Hq for one per sequence and head). */
+static double alibi_slope(const float *alibi, int stride, int b, int h)
+{
+    return (double)alibi[(size_t)b * (size_t)stride + (size_t)h];
+}
+
+/*
  * Prefill for an explicit list of (token, head) rows.
  *   q: [T, Hq, d]; k, v: [T, Hkv, d]; cu_seqlens: [B+1] prefix sums.
  *   rows_t/rows_h: the requested rows (nrows of them).
  *   o: [nrows, d] (double); lse: [nrows] (double).
- * Query token t of sequence b (local index i = t - cu[b]) sees keys
- * cu[b] + j for j in [0, L_b) (non-causal) or j in [0, i] (causal).
+ * Query token t of sequence b (local index i = t - cu[b]) sees the keys
+ * cu[b] + j with key_visible(i, j, ...).  softcap > 0 caps the logits;
+ * alibi (fp32, may be NULL) adds -slope * |i - j|.
  * Returns 0, or -1 on an invalid argument.
  */
-int oracle_prefill_rows(const void *q, const void *k, const void *v, int dtype,
-                        const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d,
-                        int causal, double scale, const int64_t *rows_t,
-                        const int32_t *rows_h, int64_t nrows, double *o, double *lse)
+int oracle_prefill_rows_ex(const void *q, const void *k, const void *v, int dtype,
+                           const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d,
+                           int causal, double scale, int window_left, int window_right,
+                           double softcap, const float *alibi, int alibi_stride,
+                           const int64_t *rows_t, const int32_t *rows_h, int64_t nrows,
+                           double *o, double *lse)
 {
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0)
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || softcap < 0.0 ||
+        alibi_stride < 0)
         return -1;
     int64_t T = cu_seqlens[B];
     int64_t maxlen = 0;
@@ -151,9 +206,9 @@ int oracle_prefill_rows(const void *q, const void *k, const void *v, int dtype,
         size_t cap = (size_t)(maxlen > 0 ? maxlen : 1);
         double *s = (double *)malloc(cap * sizeof(double));
         double *p = (double *)malloc(cap * sizeof(double));
+        double *bias = (double *)malloc(cap * sizeof(double));
         size_t *kr = (size_t *)malloc(cap * sizeof(size_t));
-        size_t *vr = (size_t *)malloc(cap * sizeof(size_t));
-        if (!s || !p || !kr || !vr) {
+        if (!s || !p || !bias || !kr) {
 #pragma omp atomic write
             bad = 1;
         } else {
@@ -166,31 +221,46 @@ int oracle_prefill_rows(const void *q, const void *k, const void *v, int dtype,
                 int64_t start = cu_seqlens[b];
                 int64_t L = cu_seqlens[b + 1] - start;
                 int64_t i = t - start;
-                int64_t n = causal ? i + 1 : L;
-                for (int64_t j = 0; j < n; ++j) {
-                    kr[j] = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;
-                    vr[j] = kr[j];
+                double slope = alibi ? alibi_slope(alibi, alibi_stride, b, h) : 0.0;
+                size_t n = 0;
+                for (int64_t j = 0; j < L; ++j) {
+                    if (!key_visible(i, j, L, causal, window_left, window_right))
+                        continue;
+                    kr[n] = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;
+                    bias[n] = -slope * fabs((double)(i - j));
+                    ++n;
                 }
                 size_t qrow = ((size_t)t * (size_t)Hq + (size_t)h) * (size_t)d;
-                attend_one_row(q, k, v, dtype, qrow, kr, vr, (size_t)n, d, scale, s, p,
-                               o + (size_t)r * (size_t)d, lse + r);
+                attend_one_row(q, k, v, dtype, qrow, kr, kr, n, d, scale, softcap,
+                               alibi ? bias : NULL, s, p, o + (size_t)r * (size_t)d, lse + r);
             }
         }
         free(s);
         free(p);
+        free(bias);
         free(kr);
-        free(vr);
     }
     return bad ? -1 : 0;
 }
 
+/* oracle_prefill_rows_ex with no window, cap or ALiBi. */
+int oracle_prefill_rows(const void *q, const void *k, const void *v, int dtype,
+                        const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d,
+                        int causal, double scale, const int64_t *rows_t,
+                        const int32_t *rows_h, int64_t nrows, double *o, double *lse)
+{
+    return oracle_prefill_rows_ex(q, k, v, dtype, cu_seqlens, B, Hq, Hkv, d, causal, scale,
+                                  -1, -1, 0.0, NULL, 0, rows_t, rows_h, nrows, o, lse);
+}
+
 /*
  * Full prefill: every (token, head).  o: [T, Hq, d] double; lse: [Hq, T]
- * double (may be NULL).
+ * double (may be NULL).  Variant arguments as in oracle_prefill_rows_ex.
  */
-int oracle_prefill(const void *q, const void *k, const void *v, int dtype,
-                   const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
-                   double scale, double *o, double *lse)
+int oracle_prefill_ex(const void *q, const void *k, const void *v, int dtype,
+                      const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                      double scale, int window_left, int window_right, double softcap,
+                      const float *alibi, int alibi_stride, double *o, double *lse)
 {
     if (B < 0 || Hq <= 0)
         return -1;
@@ -211,8 +281,9 @@ int oracle_prefill(const void *q, const void *k, const void *v, int dtype,
             rt[t * Hq + h] = t;
             rh[t * Hq + h] = h;
         }
-    int rc = oracle_prefill_rows(q, k, v, dtype, cu_seqlens, B, Hq, Hkv, d, causal, scale,
-                                 rt, rh, nrows, o, l);
+    int rc = oracle_prefill_rows_ex(q, k, v, dtype, cu_seqlens, B, Hq, Hkv, d, causal, scale,
+                                    window_left, window_right, softcap, alibi, alibi_stride,
+                                    rt, rh, nrows, o, l);
     if (rc == 0 && lse)
         for (int64_t t = 0; t < T; ++t)
             for (int h = 0; h < Hq; ++h)
@@ -223,43 +294,72 @@ int oracle_prefill(const void *q, const void *k, const void *v, int dtype,
     return rc;
 }
 
+/* oracle_prefill_ex with no window, cap or ALiBi. */
+int oracle_prefill(const void *q, const void *k, const void *v, int dtype,
+                   const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                   double scale, double *o, double *lse)
+{
+    return oracle_prefill_ex(q, k, v, dtype, cu_seqlens, B, Hq, Hkv, d, causal, scale, -1, -1,
+                             0.0, NULL, 0, o, lse);
+}
+
 /*
  * The probability matrix P of one (sequence, head) for small cases:
  * P: [L, L] double, row i = query i, column j = key j, zero where masked.
+ * Variant arguments as in oracle_prefill_rows_ex.
  */
 int oracle_prefill_probs(const void *q, const void *k, int dtype, const int32_t *cu_seqlens,
-                         int B, int Hq, int Hkv, int d, int causal, double scale, int b,
-                         int h, double *P)
+                         int B, int Hq, int Hkv, int d, int causal, double scale,
+                         int window_left, int window_right, double softcap, const float *alibi,
+                         int alibi_stride, int b, int h, double *P)
 {
-    if (b < 0 || b >= B || h < 0 || h >= Hq || Hq % Hkv != 0)
+    if (b < 0 || b >= B || h < 0 || h >= Hq || Hq % Hkv != 0 || softcap < 0.0)
         return -1;
     int64_t start = cu_seqlens[b];
     int64_t L = cu_seqlens[b + 1] - start;
     int kh = h / (Hq / Hkv);
-    double *s = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
-    if (!s)
+    size_t cap = (size_t)(L > 0 ? L : 1);
+    double *s = (double *)malloc(cap * sizeof(double));
+    double *bias = (double *)malloc(cap * sizeof(double));
+    size_t *kr = (size_t *)malloc(cap * sizeof(size_t));
+    int64_t *col = (int64_t *)malloc(cap * sizeof(int64_t));
+    if (!s || !bias || !kr || !col) {
+        free(s);
+        free(bias);
+        free(kr);
+        free(col);
         return -1;
+    }
+    double slope = alibi ? alibi_slope(alibi, alibi_stride, b, h) : 0.0;
     for (int64_t i = 0; i < L; ++i) {
-        int64_t n = causal ? i + 1 : L;
-        size_t qrow = ((size_t)(start + i) * (size_t)Hq + (size_t)h) * (size_t)d;
-        for (int64_t j = 0; j < n; ++j) {
-            size_t krow = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;
-            double dot = 0.0;
-            for (int c = 0; c < d; ++c)
-                dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krow + (size_t)c, dtype);
-            s[j] = scale * dot;
+        size_t n = 0;
+        for (int64_t j = 0; j < L; ++j) {
+            P[(size_t)i * (size_t)L + (size_t)j] = 0.0;
+            if (!key_visible(i, j, L, causal, window_left, window_right))
+                continue;
+            kr[n] = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;
+            bias[n] = -slope * fabs((double)(i - j));
+            col[n] = j;
+            ++n;
         }
+        if (n == 0)
+            continue;
+        size_t qrow = ((size_t)(start + i) * (size_t)Hq + (size_t)h) * (size_t)d;
+        row_logits(q, k, dtype, qrow, kr, n, d, scale, softcap, alibi ? bias : NULL, s);
         double m = s[0];
-        for (int64_t j = 1; j < n; ++j)
+        for (size_t j = 1; j < n; ++j)
             if (s[j] > m)
                 m = s[j];
         double z = 0.0;
-        for (int64_t j = 0; j < n; ++j)
+        for (size_t j = 0; j < n; ++j)
             z += exp(s[j] - m);
-        for (int64_t j = 0; j < L; ++j)
-            P[(size_t)i * (size_t)L + (size_t)j] = (j < n) ? exp(s[j] - m) / z : 0.0;
+        for (size_t j = 0; j < n; ++j)
+            P[(size_t)i * (size_t)L + (size_t)col[j]] = exp(s[j] - m) / z;
     }
     free(s);
+    free(bias);
+    free(kr);
+    free(col);
     return 0;
 }
 
@@ -320,7 +420,8 @@ int oracle_decode_paged(const void *q, const void *k_pages, const void *v_pages,
                 }
                 double l;
                 attend_one_row(q, k_pages, v_pages, dtype, (size_t)r * (size_t)d, kr, kr,
-                               (size_t)n, d, scale, s, p, o + (size_t)r * (size_t)d, &l);
+                               (size_t)n, d, scale, 0.0, NULL, s, p, o + (size_t)r * (size_t)d,
+                               &l);
                 if (lse)
                     lse[r] = l;
             }

@@ -16,16 +16,17 @@ import pytest
 from oracle import build as oracle_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_variant_pins.py")]
 
 MUTANTS = {
     "scale_dropped": ("s[j] = scale * dot;", "s[j] = dot;"),
-    "causal_excludes_diagonal": ("int64_t n = causal ? i + 1 : L;", "int64_t n = causal ? i : L;"),
+    "causal_excludes_diagonal": ("if (causal && j > i)", "if (causal && j >= i)"),
     "gqa_head_modulo": ("int kh = h / group;\n", "int kh = h % Hkv;\n"),
     "lse_without_max": ("*lse_out = m + log(z);", "*lse_out = log(z);"),
     "no_normalisation": ("p[j] = p[j] / z;", "p[j] = p[j];"),
-    "scores_use_values": ("dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);",
-                          "dot += elem(q, qrow + (size_t)c, dtype) * elem(v, krows[j] + (size_t)c, dtype);"),
+    "scores_transposed_operands": ("dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);",
+                                   "dot += elem(q, krows[j] + (size_t)c, dtype) * elem(k, qrow + (size_t)c, dtype);"),
     "exp_sign_flipped": ("p[j] = exp(s[j] - m);", "p[j] = exp(m - s[j]);"),
     "wrong_query_head": ("size_t qrow = ((size_t)t * (size_t)Hq + (size_t)h) * (size_t)d;",
                          "size_t qrow = ((size_t)t * (size_t)Hq + (size_t)(Hq - 1 - h)) * (size_t)d;"),
@@ -33,8 +34,29 @@ MUTANTS = {
     "decode_drops_last_token": ("int64_t n = seq_lens[b];", "int64_t n = seq_lens[b] - (seq_lens[b] > 1);"),
     "values_reversed": ("acc += p[j] * elem(v, vrows[j] + (size_t)c, dtype);",
                         "acc += p[j] * elem(v, vrows[n - 1 - j] + (size_t)c, dtype);"),
-    "keys_ignore_sequence_start": ("kr[j] = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;",
-                                   "kr[j] = ((size_t)(j) * (size_t)Hkv + (size_t)kh) * (size_t)d;"),
+    "keys_ignore_sequence_start": ("kr[n] = ((size_t)(start + j) * (size_t)Hkv + (size_t)kh) * (size_t)d;",
+                                   "kr[n] = ((size_t)(j) * (size_t)Hkv + (size_t)kh) * (size_t)d;"),
+    # mask variants (skill page, section 3.3)
+    "window_left_off_by_one": ("if (window_left >= 0 && j < i - window_left)",
+                               "if (window_left >= 0 && j <= i - window_left)"),
+    "window_right_off_by_one": ("if (window_right >= 0 && j > i + window_right)",
+                                "if (window_right >= 0 && j > i + window_right + 1)"),
+    "window_sides_swapped": ("if (window_left >= 0 && j < i - window_left)",
+                             "if (window_right >= 0 && j < i - window_right)"),
+    "softcap_without_outer_factor": ("s[j] = softcap * tanh(s[j] / softcap);",
+                                     "s[j] = tanh(s[j] / softcap);"),
+    "softcap_before_scale": ("s[j] = scale * dot;\n        if (softcap > 0.0)\n            s[j] = softcap * tanh(s[j] / softcap);",
+                             "s[j] = dot;\n        if (softcap > 0.0)\n            s[j] = softcap * tanh(s[j] / softcap);\n        s[j] *= scale;"),
+    "alibi_sign_flipped": ("bias[n] = -slope * fabs((double)(i - j));",
+                                 "bias[n] = slope * fabs((double)(i - j));"),
+    "alibi_without_abs": ("bias[n] = -slope * fabs((double)(i - j));",
+                          "bias[n] = -slope * ((double)(i - j));"),
+    "alibi_slope_of_kv_head": ("double slope = alibi ? alibi_slope(alibi, alibi_stride, b, h) : 0.0;",
+                               "double slope = alibi ? alibi_slope(alibi, alibi_stride, b, kh) : 0.0;"),
+    "alibi_batch_rows_ignored": ("return (double)alibi[(size_t)b * (size_t)stride + (size_t)h];",
+                                 "return (double)alibi[(size_t)h];"),
+    "alibi_before_cap": ("        if (softcap > 0.0)\n            s[j] = softcap * tanh(s[j] / softcap);\n        if (bias)\n            s[j] += bias[j];",
+                         "        if (bias)\n            s[j] += bias[j];\n        if (softcap > 0.0)\n            s[j] = softcap * tanh(s[j] / softcap);"),
 }
 
 
@@ -54,7 +76,7 @@ def test_pins_reject_mutant(name, source, tmp_path):
     src.write_text(source.replace(old, new, 1))
     lib = oracle_build.compile_oracle(str(src), str(tmp_path / "liboracle_mutant.so"))
     env = dict(os.environ, ORACLE_LIB=lib, OMP_NUM_THREADS="2")
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", PINS],
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", *PINS],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins accepted mutant {name}:\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout, r.stdout[-2000:]
