@@ -86,9 +86,29 @@ def max_over_ranks(dist, value: float, device=None) -> float:
 # --------------------------------------------------------------------------
 # workload accounting
 # --------------------------------------------------------------------------
-def prefill_flops(lengths, Hq, d, causal=True) -> float:
-    pairs = sum(L * (L + 1) // 2 if causal else L * L for L in lengths)
+def visible_pairs(L: int, causal: bool, window=(-1, -1)) -> int:
+    """(query, key) pairs of one sequence that the mask leaves visible: key j
+    for query i when j <= i (causal) and i - left <= j <= i + right (window;
+    negative = unlimited).  Only these count as work."""
+    left, right = int(window[0]), int(window[1])
+    if left < 0 and (right < 0 or causal):
+        return L * (L + 1) // 2 if causal else L * L
+    import numpy as np
+    i = np.arange(L, dtype=np.int64)
+    lo = np.maximum(0, i - left) if left >= 0 else np.zeros_like(i)
+    r = 0 if causal else right
+    hi = np.minimum(L - 1, i + r) if r >= 0 else np.full_like(i, L - 1)
+    return int(np.maximum(0, hi - lo + 1).sum())
+
+
+def prefill_flops(lengths, Hq, d, causal=True, window=(-1, -1)) -> float:
+    pairs = sum(visible_pairs(L, causal, window) for L in lengths)
     return 4.0 * d * Hq * pairs
+
+
+def variant_of(pin) -> dict:
+    """Mask-variant arguments of a prefill workload (window, softcap, ALiBi)."""
+    return dict(pin.meta.get("variant", {})) if pin is not None else {}
 
 
 def decode_bytes(inp) -> float:
@@ -205,17 +225,17 @@ def oracle_prefill_sample(pin, n_pairs: int):
     import numpy as np
 
     import oracle
-    L = pin.lengths[0]
+    var = variant_of(pin)
     rt, rh, flops = [], [], 0.0
     pairs = [(b, h) for b in range(pin.B) for h in range(pin.Hq)][:n_pairs]
     for b, h in pairs:
-        start = int(pin.cu_seqlens[b])
+        start, L = int(pin.cu_seqlens[b]), pin.lengths[b]
         rt.extend(range(start, start + L))
         rh.extend([h] * L)
-        flops += prefill_flops([L], 1, pin.d, pin.causal)
+        flops += prefill_flops([L], 1, pin.d, pin.causal, var.get("window", (-1, -1)))
     t0 = time.perf_counter()
     oracle.prefill_rows(pin.q, pin.k, pin.v, pin.cu_seqlens, pin.causal, pin.scale,
-                        np.array(rt), np.array(rh))
+                        np.array(rt), np.array(rh), **var)
     return flops, time.perf_counter() - t0
 
 
@@ -266,6 +286,9 @@ WORKLOAD_NAMES = {
     "varlen_gqa_prefill": inputs.WORKLOADS["varlen_gqa_prefill"],
     "paged_decode": inputs.WORKLOADS["paged_decode"],
     "long_decode": inputs.WORKLOADS["long_decode"],
+    "window_prefill": inputs.WORKLOADS["window_prefill"],
+    "softcap_prefill": inputs.WORKLOADS["softcap_prefill"],
+    "alibi_prefill": inputs.WORKLOADS["alibi_prefill"],
 }
 
 
@@ -279,6 +302,8 @@ def make_workload(name):
         din = inputs.paged_decode()
     if name == "long_decode":
         din = inputs.long_decode()
+    if name in ("window_prefill", "softcap_prefill", "alibi_prefill"):
+        pin = getattr(inputs, name)()
     return pin, din
 
 
@@ -293,6 +318,9 @@ class DeviceWorkload:
             self.o = torch.empty_like(self.q)
             self.lse = torch.empty(pin.Hq, pin.T, dtype=torch.float32, device=dev)
             self.max_len = max(pin.lengths)
+            self.variant = variant_of(pin)
+            if self.variant.get("alibi_slopes") is not None:
+                self.variant["alibi_slopes"] = self.variant["alibi_slopes"].to(dev)
         if din is not None:
             self.dq, self.kp, self.vp = (t.to(dev) for t in (din.q, din.k_pages, din.v_pages))
             self.bt, self.sl = din.block_table.to(dev), din.seq_lens.to(dev)
@@ -313,7 +341,7 @@ class DeviceWorkload:
 
     def prefill(self):
         api.fa_prefill(self.q, self.k, self.v, self.o, self.lse, self.cu, self.pin.causal,
-                       self.pin.scale, self.max_len)
+                       self.pin.scale, self.max_len, **self.variant)
 
     def decode(self):
         api.fa_decode_paged(self.dq, self.kp, self.vp, self.bt, self.sl, 0, self.do,
@@ -445,7 +473,8 @@ def run_gpu(args, world, rank, local):
 
     parts, line = {}, {}
     if pin is not None:
-        fl = prefill_flops(pin.lengths, pin.Hq, pin.d, pin.causal)
+        fl = prefill_flops(pin.lengths, pin.Hq, pin.d, pin.causal,
+                           variant_of(pin).get("window", (-1, -1)))
         tf = world * fl / (pre_ms * 1e-3) / 1e12
         parts["prefill"] = {
             "workload": pin.name, "value": round(tf, 2), "unit": "TFLOP/s",

@@ -43,6 +43,7 @@ def load_library(path: str = LIB_PATH):
     lib = ctypes.CDLL(path)
     vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, i32]
+    lib.fa_prefill_ex.argtypes = lib.fa_prefill.argtypes + [i32, i32, f32, vp, i32]
     lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32, i32, i32,
                                     i32, f32, vp, vp, sz]
     lib.fa_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32,
@@ -58,7 +59,7 @@ def load_library(path: str = LIB_PATH):
     lib.fa_get_error_string.argtypes = [i32]
     lib.fa_get_error_string.restype = ctypes.c_char_p
     lib.fa_version.argtypes = []
-    for f in (lib.fa_prefill, lib.fa_decode_paged, lib.fa_decode_auto_splits, lib.fa_prefill_f32,
+    for f in (lib.fa_prefill, lib.fa_prefill_ex, lib.fa_decode_paged, lib.fa_decode_auto_splits, lib.fa_prefill_f32,
               lib.fa_decode_paged_f32, lib.fa_get_device_error, lib.fa_version):
         f.restype = ctypes.c_int
     _lib = lib
@@ -103,12 +104,17 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
 # prefill
 # --------------------------------------------------------------------------
 def fa_prefill(q, k, v, o, lse, cu_seqlens, causal: bool, scale: float = 0.0,
-               max_seqlen: int | None = None, stream=None, *, _f32: bool = False) -> None:
-    """Calls ``fa_prefill`` (bf16) or ``fa_prefill_f32`` on torch CUDA tensors.
+               max_seqlen: int | None = None, stream=None, *, window=(-1, -1),
+               softcap: float = 0.0, alibi_slopes: torch.Tensor | None = None,
+               _f32: bool = False) -> None:
+    """Calls ``fa_prefill`` / ``fa_prefill_ex`` (bf16) or ``fa_prefill_f32``
+    on torch CUDA tensors.
 
     q [T, Hq, d], k/v [T, Hkv, d], o [T, Hq, d], lse [Hq, T] fp32 or None,
     cu_seqlens int32 [B+1].  ``max_seqlen`` bounds every sequence length
-    (defaults to T, which needs no device read).
+    (defaults to T, which needs no device read).  ``window`` = (left, right)
+    (negative = unlimited), ``softcap`` (0 = off) and ``alibi_slopes``
+    (fp32 CUDA [Hq] or [B, Hq]) select the mask variants of ``fa_prefill_ex``.
     """
     dt = torch.float32 if _f32 else torch.bfloat16
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
@@ -124,18 +130,42 @@ def fa_prefill(q, k, v, o, lse, cu_seqlens, causal: bool, scale: float = 0.0,
         raise ValueError("lse must be [Hq, T]")
     B = cu_seqlens.numel() - 1
     ms = T if max_seqlen is None else int(max_seqlen)
-    fn = load_library().fa_prefill_f32 if _f32 else load_library().fa_prefill
-    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), B, Hq, Hkv, d,
-              int(bool(causal)), float(scale), _stream(stream), T, ms),
-           "fa_prefill_f32" if _f32 else "fa_prefill")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), B, Hq, Hkv, d,
+            int(bool(causal)), float(scale), _stream(stream), T, ms)
+    left, right = int(window[0]), int(window[1])
+    plain = left < 0 and right < 0 and softcap == 0 and alibi_slopes is None
+    if _f32:
+        if not plain:
+            raise ValueError("the fp32 debug path has no mask variants")
+        _check(load_library().fa_prefill_f32(*args), "fa_prefill_f32")
+        return
+    if plain:
+        _check(load_library().fa_prefill(*args), "fa_prefill")
+        return
+    stride = 0
+    if alibi_slopes is not None:
+        if alibi_slopes.dim() == 1:
+            _need(alibi_slopes, "alibi_slopes", torch.float32, 1)
+            if alibi_slopes.shape[0] != Hq:
+                raise ValueError("alibi_slopes must be [Hq] or [B, Hq]")
+        else:
+            _need(alibi_slopes, "alibi_slopes", torch.float32, 2)
+            if tuple(alibi_slopes.shape) != (B, Hq):
+                raise ValueError("alibi_slopes must be [Hq] or [B, Hq]")
+            stride = Hq
+    _check(load_library().fa_prefill_ex(*args, left, right, float(softcap), _ptr(alibi_slopes),
+                                        stride), "fa_prefill_ex")
 
 
 def prefill(q, k, v, cu_seqlens, causal: bool = True, scale: float = 0.0,
-            max_seqlen: int | None = None, return_lse: bool = True, stream=None):
-    """Allocates O (and LSE) and runs ``fa_prefill``.  Returns (o, lse or None)."""
+            max_seqlen: int | None = None, return_lse: bool = True, stream=None, *,
+            window=(-1, -1), softcap: float = 0.0, alibi_slopes: torch.Tensor | None = None):
+    """Allocates O (and LSE) and runs ``fa_prefill`` (``fa_prefill_ex`` when a
+    mask variant is given).  Returns (o, lse or None)."""
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device) if return_lse else None
-    fa_prefill(q, k, v, o, lse, cu_seqlens, causal, scale, max_seqlen, stream)
+    fa_prefill(q, k, v, o, lse, cu_seqlens, causal, scale, max_seqlen, stream, window=window,
+               softcap=softcap, alibi_slopes=alibi_slopes)
     return o, lse
 
 

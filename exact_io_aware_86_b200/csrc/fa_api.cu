@@ -86,10 +86,21 @@ bool set_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
-template <int D>
+// Mask variants after normalisation: window bounds -1 (no limit) or in
+// [0, max_seqlen), right bound 0 under the causal mask.
+struct Variant {
+  int wl = -1, wr = -1;
+  float softcap = 0.f;
+  const float* alibi = nullptr;
+  int alibi_stride = 0;
+  // anything beyond the plain causal (wr = 0) or full (wr = -1) mask
+  bool general() const { return softcap > 0.f || alibi != nullptr || wl >= 0 || wr > 0; }
+};
+
+template <int D, bool GENERAL>
 fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                          const int32_t* cu, int B, int Hq, int Hkv, int causal, float scale,
-                         cudaStream_t stream, int T, int max_seqlen) {
+                         cudaStream_t stream, int T, int max_seqlen, const Variant& var) {
   using namespace fa::prefill;
   CUtensorMap tq, tk, tv;
   const cuuint32_t box[2] = {64, (cuuint32_t)BM};
@@ -116,6 +127,12 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   p.causal = causal ? 1 : 0;
   p.scale_log2 = resolve_scale(scale, D) * kLog2e;
   p.num_levels = (max_seqlen + ROWS_PER_ITEM - 1) / ROWS_PER_ITEM;
+  p.wl = var.wl;
+  p.wr = var.wr;
+  p.cap_out = var.softcap > 0.f ? var.softcap * kLog2e : 0.f;
+  p.cap_in = var.softcap > 0.f ? 2.f * kLog2e * resolve_scale(scale, D) / var.softcap : 0.f;
+  p.alibi = var.alibi;
+  p.alibi_stride = var.alibi_stride;
 
   const int sms = num_sms_current();
   if (sms <= 0) return FA_ERR_CUDA;
@@ -126,17 +143,17 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   if (grid > 0x7fffffff) return FA_ERR_UNSUPPORTED;
 
   const int smem = smem_bytes<D>();
-  static bool attr_ok = set_smem(prefill_kernel<D>, smem);
+  static bool attr_ok = set_smem(prefill_kernel<D, GENERAL>, smem);
   if (!attr_ok) return FA_ERR_CUDA;
   // The kernel hands registers between its warpgroups with setmaxnreg; the
   // split only fits if the launch allots kRegsLaunch registers per thread
   // (otherwise setmaxnreg.inc could never be satisfied).
   static int launch_regs = [] {
     cudaFuncAttributes a;
-    return cudaFuncGetAttributes(&a, prefill_kernel<D>) == cudaSuccess ? a.numRegs : -1;
+    return cudaFuncGetAttributes(&a, prefill_kernel<D, GENERAL>) == cudaSuccess ? a.numRegs : -1;
   }();
   if (launch_regs < (int)kRegsLaunch) return FA_ERR_UNSUPPORTED;
-  prefill_kernel<D><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, GENERAL><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -259,15 +276,28 @@ fa_status launch_decode(const void* q, const void* kp, const void* vp, const int
 
 extern "C" {
 
-fa_status fa_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
-                     const int32_t* cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
-                     float scale, fa_stream_t stream, int total_tokens, int max_seqlen) {
+fa_status fa_prefill_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int32_t* cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                        float scale, fa_stream_t stream, int total_tokens, int max_seqlen,
+                        int window_left, int window_right, float softcap,
+                        const float* alibi_slopes, int alibi_batch_stride) {
   if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_INVALID_ARG;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0 || max_seqlen < 0)
     return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(cu_seqlens, 4) || (lse && !aligned(lse, 4)))
+      !aligned(cu_seqlens, 4) || (lse && !aligned(lse, 4)) ||
+      (alibi_slopes && !aligned(alibi_slopes, 4)))
     return FA_ERR_INVALID_ARG;
+  if (!(softcap >= 0.f) || std::isinf(softcap) || alibi_batch_stride < 0)
+    return FA_ERR_INVALID_ARG;
+  Variant var;
+  // a bound at least max_seqlen can never cut a sequence: no limit
+  var.wl = (window_left < 0 || window_left >= max_seqlen) ? -1 : window_left;
+  var.wr = causal ? 0 : ((window_right < 0 || window_right >= max_seqlen) ? -1 : window_right);
+  if (var.wr == 0) causal = 1;  // a right bound of 0 is the causal mask
+  var.softcap = softcap;
+  var.alibi = alibi_slopes;
+  var.alibi_stride = alibi_slopes ? alibi_batch_stride : 0;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (Hq > 0xFFFF) return FA_ERR_UNSUPPORTED;
   if ((long long)(max_seqlen + fa::prefill::ROWS_PER_ITEM - 1) / fa::prefill::ROWS_PER_ITEM >
@@ -275,11 +305,23 @@ fa_status fa_prefill(const void* q, const void* k, const void* v, void* o, float
     return FA_ERR_UNSUPPORTED;
   if (B == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool gen = var.general();
   if (d == 64)
-    return launch_prefill<64>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
-                              total_tokens, max_seqlen);
-  return launch_prefill<128>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
-                             total_tokens, max_seqlen);
+    return gen ? launch_prefill<64, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
+                                          s, total_tokens, max_seqlen, var)
+               : launch_prefill<64, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
+                                           scale, s, total_tokens, max_seqlen, var);
+  return gen ? launch_prefill<128, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
+                                         s, total_tokens, max_seqlen, var)
+             : launch_prefill<128, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
+                                          s, total_tokens, max_seqlen, var);
+}
+
+fa_status fa_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const int32_t* cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                     float scale, fa_stream_t stream, int total_tokens, int max_seqlen) {
+  return fa_prefill_ex(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, d, causal, scale, stream,
+                       total_tokens, max_seqlen, -1, -1, 0.f, nullptr, 0);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int d, int num_splits) {

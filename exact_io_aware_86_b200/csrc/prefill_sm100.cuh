@@ -39,6 +39,20 @@
 // fourth, which balances the two units.  P is rounded to bf16 for the MMA;
 // O is divided by the sum of those rounded values (so O is a weighted mean
 // with exactly the weights used) and the LSE uses the unrounded sum.
+//
+// Mask variants ("flash-attention" skill page, section 3.3), compiled into a
+// second instantiation (GENERAL = true) so the plain causal / full kernel
+// keeps its lean inner loop:
+//   - sliding window (left, right): query i sees keys i-left .. i+right.
+//     Each query tile visits only the K/V tiles that intersect its band
+//     [lo, hi), so a long sequence costs O(L * window), not O(L^2);
+//   - softcap c: the logit x = scale * q.k becomes c * tanh(x / c), with
+//     tanh(y) = 1 - 2 / (1 + e^(2y)) from one MUFU exp2 and one MUFU
+//     reciprocal (absolute error a few fp32 ulps of 1, times c);
+//   - ALiBi: the capped logit gets -slope * |i - j|, one FMA per score.
+// In this form a row can see no key at all in its first K/V tile (the band
+// starts inside the tile), so its running max may start at -inf; the exp
+// argument and the rescale factor are guarded for that.
 #pragma once
 
 #include "ptx.cuh"
@@ -105,7 +119,42 @@ struct Params {
   int causal;
   float scale_log2;  // softmax scale * log2(e)
   int num_levels;    // ceil(max_seqlen / 256)
+  // key band of query i: [i - wl, i + wr]; -1 = no limit on that side;
+  // wr = 0 under the causal mask.  Every kernel instantiation honours the
+  // band's tile range; only GENERAL masks inside tiles by wl / wr.
+  int wl, wr;
+  float cap_in;         // 2 * log2(e) * scale / softcap (GENERAL, softcap > 0)
+  float cap_out;        // softcap * log2(e); 0 = no softcap
+  const float* alibi;   // ALiBi slopes (GENERAL), or null
+  int alibi_stride;     // slope of (b, h) = alibi[b * alibi_stride + h]
 };
+
+// K/V tiles [lo, hi) that a query tile starting at local row rs (< len)
+// has to visit: the tiles intersecting the union of its rows' key bands.
+__device__ __forceinline__ void tile_kv_range(const Params& p, int rs, int len, int& lo, int& hi) {
+  const int nkv = (len + BN - 1) / BN;
+  const int re = min(rs + BM, len) - 1;  // last row of the tile
+  hi = p.wr >= 0 ? min(nkv, (re + p.wr) / BN + 1) : nkv;
+  lo = p.wl >= 0 ? max(0, rs - p.wl) / BN : 0;
+}
+
+// K/V tiles a work item (query tiles q0 and q0 + BM) streams: [lo, hi).  The
+// second tile's range starts no earlier and ends no earlier than the first's
+// and the two overlap or touch, so the union is one interval.
+__device__ __forceinline__ void item_kv_range(const Params& p, int q0, int len, int& lo, int& hi) {
+  tile_kv_range(p, q0, len, lo, hi);
+  if (q0 + BM < len) {
+    int lo1, hi1;
+    tile_kv_range(p, q0 + BM, len, lo1, hi1);
+    hi = max(hi, hi1);
+  }
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 // Length of sequence b as the kernel uses it: an inconsistent cu_seqlens
 // entry reports a bounds error and makes the sequence empty.
@@ -153,7 +202,7 @@ __device__ void decode_item(const Params& p, const Shared& sh, int w, int& b, in
   }
 }
 
-template <int D>
+template <int D, bool GENERAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -261,13 +310,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int start, len;
         seq_range(p, b, start, len);
         const int q0 = level * ROWS_PER_ITEM;
-        const int nkv_total = (len + BN - 1) / BN;
-        int nmax = 0;
-#pragma unroll
-        for (int t = 0; t < NQT; ++t) {
-          const int rs = q0 + t * BM;
-          if (rs < len) nmax = p.causal ? min(nkv_total, rs / BN + 1) : nkv_total;
-        }
+        int jlo, jhi;
+        item_kv_range(p, q0, len, jlo, jhi);
+        const int njobs = jhi - jlo;  // K/V tiles of this item
         const int kh = h / p.group;
         // K/V tile loads of this item; the first pair goes out before the
         // wait for the Q buffer, so it overlaps the previous item's tail
@@ -282,12 +327,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int pn = 0; pn < C::PANELS; ++pn)
               tma_load_2d(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot], kh * D + pn * 64,
-                          start + (next >> 1) * BN);
+                          start + (jlo + (next >> 1)) * BN);
             ++kv_it;
           }
           return true;
         };
-        if (!issue_kv(min(2, 2 * nmax))) break;
+        if (!issue_kv(min(2, 2 * njobs))) break;
         if (it + 1 < num_items) {
           // the next item's Q tiles come from DRAM; pull them into L2 now so
           // their load at the next item boundary is short
@@ -310,7 +355,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full,
                         h * D + pn * 64, start + q0 + t * BM);
         ++q_it;
-        if (!issue_kv(2 * nmax)) break;
+        if (!issue_kv(2 * njobs)) break;
       }
       // Before the CTA can exit, every load issued must have landed (bounded
       // wait that ignores the abort flag: the copies finish on their own).
@@ -361,55 +406,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         seq_range(p, b, start, len);
         (void)start;
         const int q0 = level * ROWS_PER_ITEM;
-        const int nkv_total = (len + BN - 1) / BN;
-        const int n0 = q0 < len ? (p.causal ? min(nkv_total, q0 / BN + 1) : nkv_total) : 0;
-        const int n1 = q0 + BM < len ? (p.causal ? min(nkv_total, (q0 + BM) / BN + 1) : nkv_total) : 0;
-        const int nmax = max(n0, n1);
+        // K/V tile range of each query tile; an absent second tile gets an
+        // empty range
+        int lo0, hi0, lo1 = 0, hi1 = 0;
+        tile_kv_range(p, q0, len, lo0, hi0);
+        if (q0 + BM < len) tile_kv_range(p, q0 + BM, len, lo1, hi1);
+        const int jlo = lo0, jhi = max(hi0, hi1);
         if (!mbar_wait(&sh.q_full, q_it & 1, abort)) { ok = false; break; }
         ++q_it;
         const uint32_t base = kv_it;
-        for (int j = 0; j <= nmax; ++j) {
-          const uint32_t k_idx = base + 2 * j, v_idx = base + 2 * j - 1;
-          if (j < nmax &&
+        // step j issues P V of tile j-1 and Q K^T of tile j, per query tile
+        for (int j = jlo; j <= jhi; ++j) {
+          const uint32_t k_idx = base + 2 * (j - jlo), v_idx = k_idx - 1;
+          if (j < jhi &&
               !mbar_wait(&sh.kv_full[k_idx % C::STAGES], (k_idx / C::STAGES) & 1, abort)) {
             ok = false;
             break;
           }
-          if (j >= 1 &&
+          if (j > jlo &&
               !mbar_wait(&sh.kv_full[v_idx % C::STAGES], (v_idx / C::STAGES) & 1, abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // tile 0
-          if (j >= 1 && j - 1 < n0) {
+          // query tile 0
+          if (j > lo0 && j <= hi0) {
             if (!mbar_wait(&sh.p_full[0], p_phase0, abort)) { ok = false; break; }
             p_phase0 ^= 1;
             tc_fence_after();
-            issue_pv(0, v_idx, j == 1);
-            if (j == n0) umma_commit(&sh.o_full[0]);
+            issue_pv(0, v_idx, j == lo0 + 1);
+            if (j == hi0) umma_commit(&sh.o_full[0]);
           }
-          if (j < n0) {
+          if (j >= lo0 && j < hi0) {
             issue_s(0, k_idx);
             umma_commit(&sh.s_full[0]);
           }
-          // tile 1
-          if (j >= 1 && j - 1 < n1) {
+          // query tile 1
+          if (j > lo1 && j <= hi1) {
             if (!mbar_wait(&sh.p_full[1], p_phase1, abort)) { ok = false; break; }
             p_phase1 ^= 1;
             tc_fence_after();
-            issue_pv(1, v_idx, j == 1);
-            if (j == n1) umma_commit(&sh.o_full[1]);
+            issue_pv(1, v_idx, j == lo1 + 1);
+            if (j == hi1) umma_commit(&sh.o_full[1]);
           }
-          if (j < n1) {
+          if (j >= lo1 && j < hi1) {
             issue_s(1, k_idx);
             umma_commit(&sh.s_full[1]);
           }
-          if (j >= 1) umma_commit(&sh.kv_empty[v_idx % C::STAGES]);
-          if (j < nmax) umma_commit(&sh.kv_empty[k_idx % C::STAGES]);
-          if (j == nmax - 1 || nmax == 0) umma_commit(&sh.q_empty);  // last S of the item issued
+          if (j > jlo) umma_commit(&sh.kv_empty[v_idx % C::STAGES]);
+          if (j < jhi) umma_commit(&sh.kv_empty[k_idx % C::STAGES]);
+          if (j == jhi - 1 || jhi == jlo) umma_commit(&sh.q_empty);  // last S of the item issued
         }
-        kv_it = base + 2 * nmax;
+        kv_it = base + 2 * (jhi - jlo);
       }
       // every MMA issued must finish before TMEM is released
       umma_commit(&sh.mma_done);
@@ -436,16 +484,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       seq_range(p, b, start, len);
       const int rs = level * ROWS_PER_ITEM + t * BM;  // first row of this tile
       if (rs >= len) continue;
-      const int nkv_total = (len + BN - 1) / BN;
-      const int n = p.causal ? min(nkv_total, rs / BN + 1) : nkv_total;
+      int jlo, jhi;
+      tile_kv_range(p, rs, len, jlo, jhi);
       const int qpos = rs + row;
+      // ALiBi slope of this (sequence, head) in log2 units (GENERAL only)
+      const float slope2 =
+          (GENERAL && p.alibi) ? __ldg(p.alibi + (size_t)b * p.alibi_stride + h) * 1.4426950408889634f
+                               : 0.f;
       float m_ref = -INFINITY;
       // row sums, each as two interleaved fp32 pairs: le = exact sum of
       // exp (for the LSE), lr = sum of the bf16 values the PV MMA consumes
       // (normalises O consistently with its own weights)
       uint64_t le_a = 0, le_b = 0;
       float lr_a0 = 0.f, lr_a1 = 0.f, lr_b0 = 0.f, lr_b1 = 0.f;
-      for (int j = 0; j < n; ++j) {
+      for (int j = jlo; j < jhi; ++j) {
         if (!mbar_wait(&sh.s_full[t], s_phase, abort)) { ok = false; break; }
         s_phase ^= 1;
         tc_fence_after();
@@ -455,14 +507,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
         const int kv0 = j * BN;
-        // masking: keys past the sequence end, and (causal) keys after the query
-        if (kv0 + BN > len || (p.causal && kv0 + BN - 1 > rs)) {
-          const int lim = min(len, p.causal ? qpos + 1 : len) - kv0;  // keys [0, lim) visible
+        if constexpr (GENERAL) {
+          // logits in log2 units: optional cap, then the ALiBi distance penalty
+          if (p.cap_out > 0.f) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              s[c][e] = (c * 32 + e >= lim) ? __float_as_uint(-INFINITY) : s[c][e];
+              for (int e = 0; e < 32; ++e) {
+                // tanh(y) = 1 - 2 / (1 + 2^(2 y log2 e)); saturates to +-1
+                const float big = ex2(__uint_as_float(s[c][e]) * p.cap_in);
+                const float th = fmaf(-2.f, rcp_approx(1.f + big), 1.f);
+                s[c][e] = __float_as_uint(th * p.cap_out);
+              }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e) s[c][e] = __float_as_uint(__uint_as_float(s[c][e]) * sl);
+          }
+          if (slope2 != 0.f) {
+            const float d0 = (float)(kv0 - qpos);  // key - query for column 0
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                s[c][e] = __float_as_uint(
+                    fmaf(-slope2, fabsf(d0 + (float)(c * 32 + e)), __uint_as_float(s[c][e])));
+          }
+          // masking: keys outside [0, len) or outside the row's band
+          if (kv0 + BN > len || (p.wr >= 0 && kv0 + BN - 1 > rs + p.wr) ||
+              (p.wl >= 0 && kv0 < rs + BM - 1 - p.wl)) {
+            const int lim_lo = p.wl >= 0 ? qpos - p.wl - kv0 : -1;  // columns [lim_lo, lim_hi)
+            const int lim_hi = min(len, p.wr >= 0 ? qpos + p.wr + 1 : len) - kv0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                s[c][e] = (c * 32 + e < lim_lo || c * 32 + e >= lim_hi)
+                              ? __float_as_uint(-INFINITY) : s[c][e];
+          }
+        } else {
+          // masking: keys past the sequence end, and (causal) keys after the query
+          if (kv0 + BN > len || (p.causal && kv0 + BN - 1 > rs)) {
+            const int lim = min(len, p.causal ? qpos + 1 : len) - kv0;  // keys [0, lim) visible
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                s[c][e] = (c * 32 + e >= lim) ? __float_as_uint(-INFINITY) : s[c][e];
+          }
         }
         // row max: four independent chains of three-input maxima
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
@@ -475,14 +568,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mx2 = fmax3(mx2, __uint_as_float(s[c][e + 4]), __uint_as_float(s[c][e + 5]));
             mx3 = fmax3(mx3, __uint_as_float(s[c][e + 6]), __uint_as_float(s[c][e + 7]));
           }
-        const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
+        const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * (GENERAL ? 1.f : sl);
         float alpha = 1.f;
         bool rescale = false;
-        if (j == 0) {
-          m_ref = (mx_s == -INFINITY) ? 0.f : mx_s;
+        if (j == jlo) {
+          // GENERAL keeps -inf for a row that sees nothing in this tile
+          m_ref = (!GENERAL && mx_s == -INFINITY) ? 0.f : mx_s;
         } else if (__any_sync(0xffffffffu, mx_s > m_ref + kRescaleThreshold)) {
           const float m_new = fmaxf(m_ref, mx_s);
-          alpha = ex2(m_ref - m_new);
+          // (m_ref == m_new also covers -inf == -inf, where the difference is NaN)
+          alpha = (GENERAL && m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
           const uint64_t a2 = f2_pack(alpha, alpha);
           le_a = f2_mul(le_a, a2);
           le_b = f2_mul(le_b, a2);
@@ -495,13 +590,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         // P = 2^(s*scale*log2e - m): three of every four pairs on MUFU, one on
         // the FMA pipe; packed bf16 pairs overwrite s[c][0..15] in order
-        const uint64_t neg2 = f2_pack(-m_ref, -m_ref);
+        const float m_use = (GENERAL && m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t neg2 = f2_pack(-m_use, -m_use);
+        // GENERAL: s already holds scaled logits, so the FMA multiplies by 1
+        const uint64_t mul2 = GENERAL ? f2_pack(1.f, 1.f) : sl2;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const uint64_t x =
-                f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), sl2, neg2);
+                f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), mul2, neg2);
             uint64_t pr;
             if (((e >> 1) & 3) == 3) {
               pr = exp2_fma_pair(x);

@@ -202,7 +202,24 @@ WORKLOADS = {
     "varlen_gqa_prefill": "varlen GQA causal prefill, 8 seqs L~U[512,8192], Hq=32 Hkv=8 d=128",
     "paged_decode": "paged decode, 64 requests, Hq=32 Hkv=8 d=128, ctx~U[1024,32768], page 16",
     "long_decode": "split-KV decode, 2 requests x 131072 ctx, Hq=32 Hkv=8 d=128, page 64",
+    # mask variants of the skill page's advanced-features table (section 3.3)
+    "window_prefill": "sliding-window causal prefill, window (4096, 0), 2 seqs x 16384, "
+                      "Hq=32 Hkv=8 d=128",
+    "softcap_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 with softcap 50",
+    "alibi_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 with ALiBi slopes",
 }
+
+
+def alibi_slopes_geometric(H: int) -> torch.Tensor:
+    """fp32 [H]: the geometric slope sequence 2^(-8 (h+1) / H) that ALiBi
+    models use for H heads (H a power of two).  The pages give the ALiBi
+    argument's shape but no values; this is input data, not the method."""
+    return torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32)
+
+
+def uniform_slopes(shape, lo: float, hi: float, gen: torch.Generator) -> torch.Tensor:
+    """fp32 slopes drawn uniformly from [lo, hi)."""
+    return (torch.rand(*shape, generator=gen, dtype=torch.float32) * (hi - lo) + lo).contiguous()
 
 
 def tiny(causal: bool) -> PrefillInputs:
@@ -223,6 +240,30 @@ def varlen_gqa_prefill() -> PrefillInputs:
     return PrefillInputs(name="varlen_gqa_prefill", q=q, k=k, v=v,
                          cu_seqlens=cu_seqlens_of(lengths), lengths=lengths, causal=True,
                          scale=fp32_scale(128), meta={"seed": 1003})
+
+
+def window_prefill() -> PrefillInputs:
+    """Mistral-style sliding window (4096, 0) (skill page, section 3.3) over
+    two long sequences."""
+    inp = make_prefill([16384, 16384], 32, 8, 128, True, seed=1006, name="window_prefill")
+    inp.meta["variant"] = {"window": (4096, 0)}
+    return inp
+
+
+def softcap_prefill() -> PrefillInputs:
+    """The causal MHA workload with the page's example cap, softcap=50."""
+    inp = mha_prefill()
+    inp.name = "softcap_prefill"
+    inp.meta["variant"] = {"softcap": 50.0}
+    return inp
+
+
+def alibi_prefill() -> PrefillInputs:
+    """The causal MHA workload with one ALiBi slope per head."""
+    inp = mha_prefill()
+    inp.name = "alibi_prefill"
+    inp.meta["variant"] = {"alibi_slopes": alibi_slopes_geometric(16)}
+    return inp
 
 
 def _decode_from_lengths(name, seq_lens, page_size, seed, gen):

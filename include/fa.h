@@ -81,6 +81,38 @@ fa_status fa_prefill(const void *q, const void *k, const void *v, void *o, float
                      float scale, fa_stream_t stream, int total_tokens, int max_seqlen);
 
 /*
+ * Prefill with the mask variants of the "flash-attention" skill page,
+ * section 3.3 (advanced features).  The first fifteen arguments are those of
+ * fa_prefill; fa_prefill is this call with (-1, -1, 0, NULL, 0).
+ *
+ *   window_left,  sliding window (window_size = (left, right)): query i of a
+ *   window_right  sequence sees key j only when
+ *                 i - window_left <= j <= i + window_right; a negative value
+ *                 means no limit on that side.  causal != 0 keeps j <= i as
+ *                 well (so window_right does not matter then); (-1, 0)
+ *                 without causal is the causal mask.
+ *   softcap       > 0: every logit x = scale * <q_i, k_j> becomes
+ *                 softcap * tanh(x / softcap) (Gemma-2 style capping);
+ *                 0 = off.  Negative, NaN or infinite: FA_ERR_INVALID_ARG.
+ *   alibi_slopes  fp32, device, or NULL.  Adds -slope * |i - j| to the
+ *                 (capped) logit of query i and key j, with
+ *                 slope = alibi_slopes[b * alibi_batch_stride + h] for
+ *                 sequence b and query head h: stride 0 for one slope per
+ *                 head ([Hq]), Hq for [B, Hq].  The array must hold every
+ *                 index that formula reaches.
+ *   alibi_batch_stride  >= 0 (FA_ERR_INVALID_ARG otherwise).
+ * LSE is the log-sum-exp of the final logits (after cap and ALiBi) over the
+ * visible keys.  Every row sees at least its own key, so none is empty.  A
+ * window shorter than the sequence also cuts the work: each 128-row query
+ * tile visits only the 128-key tiles its rows' windows reach.
+ */
+fa_status fa_prefill_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                        float scale, fa_stream_t stream, int total_tokens, int max_seqlen,
+                        int window_left, int window_right, float softcap,
+                        const float *alibi_slopes, int alibi_batch_stride);
+
+/*
  * Paged decode: one query token per request at the end of its context.
  *
  *   q            bf16 [B, Hq, d]

@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("fa_prefill", "fa_decode_paged", "fa_decode_workspace_size",
+    for n in ("fa_prefill", "fa_prefill_ex", "fa_decode_paged", "fa_decode_workspace_size",
               "fa_decode_auto_splits", "fa_get_error_string", "fa_get_device_error"):
         assert n in names
 
@@ -72,6 +72,27 @@ def test_prefill_argument_checks(lib):
     # empty problems are a no-op (no launch)
     assert _prefill(lib, B=0) == api.FA_OK
     assert _prefill(lib, T=0) == api.FA_OK
+
+
+def _prefill_ex(lib, wl=-1, wr=-1, cap=0.0, alibi=None, stride=0, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, cu=FAKE, B=1, Hq=4, Hkv=2, d=128,
+             causal=1, scale=0.0, stream=None, T=16, maxlen=16)
+    a.update(kw)
+    return lib.fa_prefill_ex(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu"], a["B"], a["Hq"],
+                             a["Hkv"], a["d"], a["causal"], a["scale"], a["stream"], a["T"],
+                             a["maxlen"], wl, wr, cap, alibi, stride)
+
+
+def test_prefill_ex_argument_checks(lib):
+    assert _prefill_ex(lib, cap=-0.5) == api.FA_ERR_INVALID_ARG
+    assert _prefill_ex(lib, cap=float("nan")) == api.FA_ERR_INVALID_ARG
+    assert _prefill_ex(lib, cap=float("inf")) == api.FA_ERR_INVALID_ARG
+    assert _prefill_ex(lib, alibi=FAKE, stride=-1) == api.FA_ERR_INVALID_ARG
+    assert _prefill_ex(lib, alibi=ctypes.c_void_p(0x1002)) == api.FA_ERR_INVALID_ARG  # misaligned
+    assert _prefill_ex(lib, q=None, wl=4) == api.FA_ERR_INVALID_ARG
+    assert _prefill_ex(lib, d=96, wl=4) == api.FA_ERR_UNSUPPORTED
+    # empty problems are a no-op whatever the variant
+    assert _prefill_ex(lib, B=0, wl=3, wr=2, cap=30.0, alibi=FAKE, stride=4) == api.FA_OK
 
 
 def _decode(lib, **kw):
