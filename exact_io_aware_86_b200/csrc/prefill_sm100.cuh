@@ -418,12 +418,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // step j issues P V of tile j-1 and Q K^T of tile j, per query tile
         for (int j = jlo; j <= jhi; ++j) {
           const uint32_t k_idx = base + 2 * (j - jlo), v_idx = k_idx - 1;
-          if (j < jhi &&
+          // both slots are normally full already: test them together so the
+          // two barrier latencies overlap, and block only on a miss
+          const bool k_ready = j >= jhi || mbar_try_wait(smem_u32(&sh.kv_full[k_idx % C::STAGES]),
+                                                         (k_idx / C::STAGES) & 1);
+          const bool v_ready = j <= jlo || mbar_try_wait(smem_u32(&sh.kv_full[v_idx % C::STAGES]),
+                                                         (v_idx / C::STAGES) & 1);
+          if (!k_ready &&
               !mbar_wait(&sh.kv_full[k_idx % C::STAGES], (k_idx / C::STAGES) & 1, abort)) {
             ok = false;
             break;
           }
-          if (j > jlo &&
+          if (!v_ready &&
               !mbar_wait(&sh.kv_full[v_idx % C::STAGES], (v_idx / C::STAGES) & 1, abort)) {
             ok = false;
             break;
@@ -557,18 +563,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 s[c][e] = (c * 32 + e >= lim) ? __float_as_uint(-INFINITY) : s[c][e];
           }
         }
-        // row max: four independent chains of three-input maxima
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        // row max: eight independent chains of three-input maxima (short
+        // chains: the max is on the tile's critical path)
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int k = 0; k < 8; ++k)
+          mx[k] = fmaxf(__uint_as_float(s[k >> 1][(k & 1) * 16]), __uint_as_float(s[k >> 1][(k & 1) * 16 + 1]));
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            mx0 = fmax3(mx0, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
-            mx1 = fmax3(mx1, __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
-            mx2 = fmax3(mx2, __uint_as_float(s[c][e + 4]), __uint_as_float(s[c][e + 5]));
-            mx3 = fmax3(mx3, __uint_as_float(s[c][e + 6]), __uint_as_float(s[c][e + 7]));
-          }
-        const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * (GENERAL ? 1.f : sl);
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+          for (int e = 2; e < 16; e += 2)
+            mx[k] = fmax3(mx[k], __uint_as_float(s[k >> 1][(k & 1) * 16 + e]),
+                          __uint_as_float(s[k >> 1][(k & 1) * 16 + e + 1]));
+        const float mx_s = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
+                                 fmaxf(mx[6], mx[7])) * (GENERAL ? 1.f : sl);
         float alpha = 1.f;
         bool rescale = false;
         if (j == jlo) {
