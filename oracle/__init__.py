@@ -105,10 +105,14 @@ class Oracle:
                                              ci, ci, cd, vp, ci, ci, ci, vp]
         lib.oracle_decode_paged.argtypes = [vp, vp, vp, ci, vp, vp, ci, ci, ci, ci, ci, ci,
                                             c64, cd, vp, vp]
+        lib.oracle_rope.argtypes = [vp, ci, c64, ci, vp, vp, vp, c64, ci, ci, vp]
+        lib.oracle_decode_paged_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
+                                                   ci, c64, cd, vp, vp, c64, ci, ci, vp, vp, vp]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_set_num_threads.argtypes = [ci]
         for f in (lib.oracle_prefill_rows_ex, lib.oracle_prefill_ex, lib.oracle_prefill_probs,
-                  lib.oracle_decode_paged, lib.oracle_num_threads):
+                  lib.oracle_decode_paged, lib.oracle_num_threads, lib.oracle_rope,
+                  lib.oracle_decode_paged_append):
             f.restype = ctypes.c_int
         lib.oracle_set_num_threads.restype = None
         self._lib = lib
@@ -221,6 +225,62 @@ class Oracle:
         return o, lse
 
 
+    def rope(self, x, pos, cos, sin, rotary_dim: int, interleaved: bool = False):
+        """Exact RoPE of rows x [n, d] at positions pos [n] with fp32 tables
+        cos/sin [max_pos, rotary_dim/2].  Returns float64 [n, d] (unrounded)."""
+        xa, dt = _as_np(x)
+        n, d = xa.shape
+        ps = _int_np(pos, np.int32)
+        ca = np.ascontiguousarray(_as_np(cos)[0], dtype=np.float32)
+        sa = np.ascontiguousarray(_as_np(sin)[0], dtype=np.float32)
+        out = np.zeros((n, d), np.float64)
+        rc = self._lib.oracle_rope(_ptr(xa), dt, n, d, _ptr(ps), _ptr(ca), _ptr(sa), ca.shape[0],
+                                   int(rotary_dim), int(bool(interleaved)), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle_rope rejected its arguments (rc={rc})")
+        return out
+
+    def decode_paged_append(self, q, k_new, v_new, k_pages, v_pages, block_table, cache_seqlens,
+                            scale: float, cos=None, sin=None, rotary_dim: int | None = None,
+                            interleaved: bool = False):
+        """Append one token per request to a copy of the paged cache (with
+        RoPE when cos/sin are given) and attend.  bf16 tensors.
+
+        Returns (o [B, Hq, d] float64, lse [B, Hq] float64, k_pages, v_pages
+        (updated copies, bf16 bit patterns as uint16 arrays), q_rot [B, Hq, d]
+        float64 (the bf16-rounded rotated queries)).
+        """
+        (qa, c1), (kn, c2), (vn, c3) = _as_np(q), _as_np(k_new), _as_np(v_new)
+        (kp, c4), (vpg, c5) = _as_np(k_pages), _as_np(v_pages)
+        if {c1, c2, c3, c4, c5} != {_BF16}:
+            raise TypeError("decode_paged_append takes bf16 tensors")
+        kp, vpg = kp.copy(), vpg.copy()
+        bt = _int_np(block_table, np.int32)
+        cs = _int_np(cache_seqlens, np.int32)
+        B, Hq, d = qa.shape
+        num_pages, page_size, Hkv, _ = kp.shape
+        if cos is not None:
+            ca = np.ascontiguousarray(_as_np(cos)[0], dtype=np.float32)
+            sa = np.ascontiguousarray(_as_np(sin)[0], dtype=np.float32)
+            rd = int(rotary_dim if rotary_dim is not None else 2 * ca.shape[1])
+            mp = ca.shape[0]
+        else:
+            ca = sa = None
+            rd, mp = 0, 0
+        o = np.zeros((B, Hq, d), np.float64)
+        lse = np.zeros((B, Hq), np.float64)
+        qr = np.zeros((B, Hq, d), np.float64)
+        rc = self._lib.oracle_decode_paged_append(
+            _ptr(qa), _ptr(kn), _ptr(vn), _ptr(kp), _ptr(vpg), _ptr(bt), _ptr(cs), B, Hq, Hkv, d,
+            page_size, bt.shape[1], num_pages, float(scale), _ptr_or_null(ca), _ptr_or_null(sa),
+            mp, rd, int(bool(interleaved)), _ptr(qr), _ptr(o), _ptr(lse))
+        if rc == -2:
+            raise IndexError("a block_table entry the append or attention needs is out of the pool")
+        if rc != 0:
+            raise ValueError(f"oracle_decode_paged_append rejected its arguments (rc={rc})")
+        return o, lse, kp, vpg, qr
+
+
 _default: Oracle | None = None
 
 
@@ -251,6 +311,14 @@ def prefill_probs(*args, **kw):
 
 def decode_paged(*args, **kw):
     return default().decode_paged(*args, **kw)
+
+
+def rope(*args, **kw):
+    return default().rope(*args, **kw)
+
+
+def decode_paged_append(*args, **kw):
+    return default().decode_paged_append(*args, **kw)
 
 
 def set_num_threads(n: int) -> None:

@@ -35,6 +35,16 @@
  *    -slope * |i - j| added to the logit of query i and key j.  Logit here
  *    means the scaled score scale * <q, k>; the cap is applied first and the
  *    ALiBi penalty is added to the capped value.
+ *  - "flash-attention" skill page, section 3.5 (inference KV cache): one new
+ *    token per request is appended to the (paged) cache -- k_new and v_new go
+ *    to position cache_seqlens[b] -- and its query attends to the cache
+ *    including itself; rotary_cos / rotary_sin apply RoPE on the fly to q
+ *    and k_new at that position, pairs (x_i, x_{i + rd/2}) by default and
+ *    adjacent pairs (x_{2i}, x_{2i+1}) when rotary_interleaved; dimensions
+ *    past the rotary dimension rd are left as they are.  The cache holds
+ *    bf16, so the rotated key is the exact rotation rounded once to bf16
+ *    (nearest, ties to even), and the rotated query likewise (it feeds a
+ *    bf16 product).
  *
  * Precision: every product and sum is in double.  Inputs are read in the
  * caller's element type (bf16 bit patterns, fp32 or fp64) and upcast
@@ -74,20 +84,27 @@ static double elem(const void *base, size_t i, int dtype)
  * s_j = scale * <q, k_j>, then softcap * tanh(s_j / softcap) when
  * softcap > 0, then + bias[j] when bias is not NULL.
  */
-static void row_logits(const void *q, const void *k, int dtype, size_t qrow,
-                       const size_t *krows, size_t n, int d, double scale, double softcap,
-                       const double *bias, double *s)
+static void row_logits_q(const void *q, int qdtype, const void *k, int dtype, size_t qrow,
+                         const size_t *krows, size_t n, int d, double scale, double softcap,
+                         const double *bias, double *s)
 {
     for (size_t j = 0; j < n; ++j) {
         double dot = 0.0;
         for (int c = 0; c < d; ++c)
-            dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);
+            dot += elem(q, qrow + (size_t)c, qdtype) * elem(k, krows[j] + (size_t)c, dtype);
         s[j] = scale * dot;
         if (softcap > 0.0)
             s[j] = softcap * tanh(s[j] / softcap);
         if (bias)
             s[j] += bias[j];
     }
+}
+
+static void row_logits(const void *q, const void *k, int dtype, size_t qrow,
+                       const size_t *krows, size_t n, int d, double scale, double softcap,
+                       const double *bias, double *s)
+{
+    row_logits_q(q, dtype, k, dtype, qrow, krows, n, d, scale, softcap, bias, s);
 }
 
 /*
@@ -98,10 +115,11 @@ static void row_logits(const void *q, const void *k, int dtype, size_t qrow,
  *   softcap, bias: logit modifiers of row_logits (0 / NULL for none)
  * s and p are caller scratch of length >= n.
  */
-static void attend_one_row(const void *q, const void *k, const void *v, int dtype,
-                           size_t qrow, const size_t *krows, const size_t *vrows,
-                           size_t n, int d, double scale, double softcap, const double *bias,
-                           double *s, double *p, double *o_out, double *lse_out)
+static void attend_one_row_q(const void *q, int qdtype, const void *k, const void *v,
+                             int dtype, size_t qrow, const size_t *krows, const size_t *vrows,
+                             size_t n, int d, double scale, double softcap,
+                             const double *bias, double *s, double *p, double *o_out,
+                             double *lse_out)
 {
     if (n == 0) {
         for (int c = 0; c < d; ++c)
@@ -109,7 +127,7 @@ static void attend_one_row(const void *q, const void *k, const void *v, int dtyp
         *lse_out = -INFINITY;
         return;
     }
-    row_logits(q, k, dtype, qrow, krows, n, d, scale, softcap, bias, s);
+    row_logits_q(q, qdtype, k, dtype, qrow, krows, n, d, scale, softcap, bias, s);
     /* softmax, pass 1: the row max */
     double m = s[0];
     for (size_t j = 1; j < n; ++j)
@@ -131,6 +149,15 @@ static void attend_one_row(const void *q, const void *k, const void *v, int dtyp
         o_out[c] = acc;
     }
     *lse_out = m + log(z);
+}
+
+static void attend_one_row(const void *q, const void *k, const void *v, int dtype,
+                           size_t qrow, const size_t *krows, const size_t *vrows,
+                           size_t n, int d, double scale, double softcap, const double *bias,
+                           double *s, double *p, double *o_out, double *lse_out)
+{
+    attend_one_row_q(q, dtype, k, v, dtype, qrow, krows, vrows, n, d, scale, softcap, bias, s,
+                     p, o_out, lse_out);
 }
 
 /* Sequence index b such that cu[b] <= t < cu[b+1]; -1 if none. */
@@ -430,6 +457,211 @@ int oracle_decode_paged(const void *q, const void *k_pages, const void *v_pages,
         free(p);
         free(kr);
     }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Nearest bf16 value of a double (ties to even), as a double.  bf16 keeps 8
+ * significant bits and the fp32 exponent range; the inputs here are far
+ * from its overflow and underflow limits.
+ */
+static double round_bf16(double x)
+{
+    if (x == 0.0 || !isfinite(x))
+        return x;
+    int e;
+    double m = frexp(x, &e);         /* x = m * 2^e, 0.5 <= |m| < 1 */
+    double scaled = ldexp(m, 8);     /* 8 significant bits above the point */
+    double r = nearbyint(scaled);    /* default rounding: nearest, ties to even */
+    return ldexp(r, e - 8);
+}
+
+/* Bit pattern of the bf16 value of a double that round_bf16 already made
+ * representable. */
+static uint16_t bf16_bits(double x)
+{
+    float f = (float)x;              /* exact: x has 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+/*
+ * RoPE of one d-vector at table row `row` (cos/sin rows of rd/2 fp32
+ * values): pair i is (x_i, x_{i+rd/2}), or (x_{2i}, x_{2i+1}) when
+ * interleaved, rotated by the angle whose cosine and sine are cos[i] and
+ * sin[i]; dims >= rd are copied.  In and out are double.
+ */
+static void rope_vec(const double *x, double *out, int d, int rd, int interleaved,
+                     const float *cos_row, const float *sin_row)
+{
+    for (int c = 0; c < d; ++c)
+        out[c] = x[c];
+    for (int i = 0; i < rd / 2; ++i) {
+        int a = interleaved ? 2 * i : i;
+        int b = interleaved ? 2 * i + 1 : i + rd / 2;
+        double co = (double)cos_row[i], si = (double)sin_row[i];
+        out[a] = x[a] * co - x[b] * si;
+        out[b] = x[a] * si + x[b] * co;
+    }
+}
+
+/*
+ * RoPE of n rows: x [n, d] (dtype), pos [n], tables cos/sin [max_pos, rd/2]
+ * fp32; out [n, d] double, exact (not rounded).  Returns 0, -1 on a bad
+ * argument (rd odd or > d, or a position outside [0, max_pos)).
+ */
+int oracle_rope(const void *x, int dtype, int64_t n, int d, const int32_t *pos,
+                const float *cos_tab, const float *sin_tab, int64_t max_pos, int rotary_dim,
+                int interleaved, double *out)
+{
+    if (n < 0 || d <= 0 || rotary_dim < 0 || rotary_dim > d || rotary_dim % 2 != 0)
+        return -1;
+    double *row = (double *)malloc((size_t)d * sizeof(double));
+    if (!row)
+        return -1;
+    int bad = 0;
+    for (int64_t r = 0; r < n && !bad; ++r) {
+        if (pos[r] < 0 || pos[r] >= max_pos) {
+            bad = 1;
+            break;
+        }
+        for (int c = 0; c < d; ++c)
+            row[c] = elem(x, (size_t)r * (size_t)d + (size_t)c, dtype);
+        const float *co = cos_tab + (size_t)pos[r] * (size_t)(rotary_dim / 2);
+        const float *si = sin_tab + (size_t)pos[r] * (size_t)(rotary_dim / 2);
+        rope_vec(row, out + (size_t)r * (size_t)d, d, rotary_dim, interleaved, co, si);
+    }
+    free(row);
+    return bad ? -1 : 0;
+}
+
+/*
+ * Decode with cache append and optional RoPE, bf16 tensors only.
+ *   q [B, Hq, d]; k_new, v_new [B, Hkv, d]; k_pages, v_pages
+ *   [num_pages, page_size, Hkv, d] (bf16 bits, MODIFIED: the new token is
+ *   written at position cache_seqlens[b]); block_table [B, max_blocks];
+ *   cache_seqlens [B] = tokens already cached; cos/sin [max_pos, rd/2] fp32
+ *   or NULL (no rotation; rotary_dim ignored).
+ *   q_rot (out, may be NULL) [B, Hq, d] double: the bf16 rotated queries.
+ *   o [B, Hq, d] double; lse [B, Hq] double (may be NULL).
+ * Steps: for every request, rotate (or not) q and k_new at position
+ * pos = cache_seqlens[b], round them to bf16, write k and v_new into the
+ * page slot of pos; then every query attends to tokens [0, pos] of its
+ * request's updated cache.  Returns 0, -1 on a bad argument, -2 if a page
+ * the append or the attention needs is outside [0, num_pages).
+ */
+int oracle_decode_paged_append(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                               uint16_t *k_pages, uint16_t *v_pages,
+                               const int32_t *block_table, const int32_t *cache_seqlens, int B,
+                               int Hq, int Hkv, int d, int page_size, int max_blocks,
+                               int64_t num_pages, double scale, const float *cos_tab,
+                               const float *sin_tab, int64_t max_pos, int rotary_dim,
+                               int interleaved, double *q_rot, double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || page_size <= 0)
+        return -1;
+    if (cos_tab && (rotary_dim < 0 || rotary_dim > d || rotary_dim % 2 != 0))
+        return -1;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t pos = cache_seqlens[b];
+        if (pos < 0 || pos + 1 > (int64_t)max_blocks * page_size)
+            return -1;
+        if (cos_tab && pos >= max_pos)
+            return -1;
+        if (pos + 1 > maxlen)
+            maxlen = pos + 1;
+        for (int64_t i = 0; i <= pos / page_size; ++i) {
+            int32_t pg = block_table[(size_t)b * (size_t)max_blocks + (size_t)i];
+            if (pg < 0 || pg >= num_pages)
+                return -2;
+        }
+    }
+    const int group = Hq / Hkv;
+    double *qr = (double *)malloc((size_t)B * (size_t)Hq * (size_t)d * sizeof(double));
+    double *tmp = (double *)malloc((size_t)d * sizeof(double));
+    double *rot = (double *)malloc((size_t)d * sizeof(double));
+    if (!qr || !tmp || !rot) {
+        free(qr);
+        free(tmp);
+        free(rot);
+        return -1;
+    }
+    /* 1. rotate, round to bf16, append */
+    for (int b = 0; b < B; ++b) {
+        int64_t pos = cache_seqlens[b];
+        const float *co = cos_tab ? cos_tab + (size_t)pos * (size_t)(rotary_dim / 2) : NULL;
+        const float *si = cos_tab ? sin_tab + (size_t)pos * (size_t)(rotary_dim / 2) : NULL;
+        for (int h = 0; h < Hq; ++h) {
+            size_t off = ((size_t)b * (size_t)Hq + (size_t)h) * (size_t)d;
+            for (int c = 0; c < d; ++c)
+                tmp[c] = elem(q, off + (size_t)c, OR_BF16);
+            if (co)
+                rope_vec(tmp, rot, d, rotary_dim, interleaved, co, si);
+            else
+                memcpy(rot, tmp, (size_t)d * sizeof(double));
+            for (int c = 0; c < d; ++c)
+                qr[off + (size_t)c] = round_bf16(rot[c]);
+        }
+        int64_t page = block_table[(size_t)b * (size_t)max_blocks + (size_t)(pos / page_size)];
+        int64_t slot = pos % page_size;
+        for (int kh = 0; kh < Hkv; ++kh) {
+            size_t src = ((size_t)b * (size_t)Hkv + (size_t)kh) * (size_t)d;
+            size_t dst = (((size_t)page * (size_t)page_size + (size_t)slot) * (size_t)Hkv +
+                          (size_t)kh) * (size_t)d;
+            for (int c = 0; c < d; ++c)
+                tmp[c] = elem(k_new, src + (size_t)c, OR_BF16);
+            if (co)
+                rope_vec(tmp, rot, d, rotary_dim, interleaved, co, si);
+            else
+                memcpy(rot, tmp, (size_t)d * sizeof(double));
+            for (int c = 0; c < d; ++c) {
+                k_pages[dst + (size_t)c] = bf16_bits(round_bf16(rot[c]));
+                v_pages[dst + (size_t)c] = v_new[src + (size_t)c];
+            }
+        }
+    }
+    if (q_rot)
+        memcpy(q_rot, qr, (size_t)B * (size_t)Hq * (size_t)d * sizeof(double));
+    /* 2. attend over [0, pos] of the updated cache */
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t cap = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *s = (double *)malloc(cap * sizeof(double));
+        double *p = (double *)malloc(cap * sizeof(double));
+        size_t *kr = (size_t *)malloc(cap * sizeof(size_t));
+        if (!s || !p || !kr) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < (int64_t)B * Hq; ++r) {
+                int b = (int)(r / Hq);
+                int h = (int)(r % Hq);
+                int kh = h / group;
+                int64_t n = (int64_t)cache_seqlens[b] + 1;
+                for (int64_t t = 0; t < n; ++t) {
+                    int64_t page = block_table[(size_t)b * (size_t)max_blocks + (size_t)(t / page_size)];
+                    kr[t] = (((size_t)page * (size_t)page_size + (size_t)(t % page_size)) *
+                             (size_t)Hkv + (size_t)kh) * (size_t)d;
+                }
+                double l;
+                attend_one_row_q(qr, OR_F64, k_pages, v_pages, OR_BF16, (size_t)r * (size_t)d,
+                                 kr, kr, (size_t)n, d, scale, 0.0, NULL, s, p,
+                                 o + (size_t)r * (size_t)d, &l);
+                if (lse)
+                    lse[r] = l;
+            }
+        }
+        free(s);
+        free(p);
+        free(kr);
+    }
+    free(qr);
+    free(tmp);
+    free(rot);
     return bad ? -1 : 0;
 }
 

@@ -17,7 +17,8 @@ from oracle import build as oracle_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_variant_pins.py")]
+        os.path.join(ROOT, "tests", "test_oracle_variant_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_append_pins.py")]
 
 MUTANTS = {
     "scale_dropped": ("s[j] = scale * dot;", "s[j] = dot;"),
@@ -25,8 +26,8 @@ MUTANTS = {
     "gqa_head_modulo": ("int kh = h / group;\n", "int kh = h % Hkv;\n"),
     "lse_without_max": ("*lse_out = m + log(z);", "*lse_out = log(z);"),
     "no_normalisation": ("p[j] = p[j] / z;", "p[j] = p[j];"),
-    "scores_transposed_operands": ("dot += elem(q, qrow + (size_t)c, dtype) * elem(k, krows[j] + (size_t)c, dtype);",
-                                   "dot += elem(q, krows[j] + (size_t)c, dtype) * elem(k, qrow + (size_t)c, dtype);"),
+    "scores_transposed_operands": ("dot += elem(q, qrow + (size_t)c, qdtype) * elem(k, krows[j] + (size_t)c, dtype);",
+                                   "dot += elem(q, krows[j] + (size_t)c, qdtype) * elem(k, qrow + (size_t)c, dtype);"),
     "exp_sign_flipped": ("p[j] = exp(s[j] - m);", "p[j] = exp(m - s[j]);"),
     "wrong_query_head": ("size_t qrow = ((size_t)t * (size_t)Hq + (size_t)h) * (size_t)d;",
                          "size_t qrow = ((size_t)t * (size_t)Hq + (size_t)(Hq - 1 - h)) * (size_t)d;"),
@@ -57,6 +58,19 @@ MUTANTS = {
                                  "return (double)alibi[(size_t)h];"),
     "alibi_before_cap": ("        if (softcap > 0.0)\n            s[j] = softcap * tanh(s[j] / softcap);\n        if (bias)\n            s[j] += bias[j];",
                          "        if (bias)\n            s[j] += bias[j];\n        if (softcap > 0.0)\n            s[j] = softcap * tanh(s[j] / softcap);"),
+    # decode with cache append and RoPE (skill page, section 3.5)
+    "rope_sin_sign": ("out[a] = x[a] * co - x[b] * si;", "out[a] = x[a] * co + x[b] * si;"),
+    "rope_half_pairs_adjacent": ("int b = interleaved ? 2 * i + 1 : i + rd / 2;",
+                                 "int b = interleaved ? 2 * i + 1 : i + 1;"),
+    "rope_interleaved_pairs_half": ("int a = interleaved ? 2 * i : i;", "int a = i;"),
+    "append_one_slot_late": ("int64_t slot = pos % page_size;", "int64_t slot = (pos + 1) % page_size;"),
+    "append_not_attended": ("int64_t n = (int64_t)cache_seqlens[b] + 1;",
+                            "int64_t n = (int64_t)cache_seqlens[b] + (cache_seqlens[b] == 0);"),
+    "query_not_rotated": ("            if (co)\n                rope_vec(tmp, rot, d, rotary_dim, interleaved, co, si);\n            else\n                memcpy(rot, tmp, (size_t)d * sizeof(double));\n            for (int c = 0; c < d; ++c)\n                qr[",
+                          "            memcpy(rot, tmp, (size_t)d * sizeof(double));\n            for (int c = 0; c < d; ++c)\n                qr["),
+    "value_rotated_like_key": ("v_pages[dst + (size_t)c] = v_new[src + (size_t)c];",
+                               "v_pages[dst + (size_t)c] = bf16_bits(round_bf16(rot[c]));"),
+    "bf16_rounding_truncates": ("double r = nearbyint(scaled);", "double r = trunc(scaled);"),
 }
 
 
