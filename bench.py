@@ -111,14 +111,28 @@ def variant_of(pin) -> dict:
     return dict(pin.meta.get("variant", {})) if pin is not None else {}
 
 
+def is_append(inp) -> bool:
+    return isinstance(inp, inputs.AppendInputs)
+
+
 def decode_bytes(inp) -> float:
     """Algorithmic bytes of one decode call: K and V of every context token,
-    q and o, the used block-table entries and seq_lens."""
-    ctx = [int(x) for x in inp.seq_lens]
+    q and o, the used block-table entries and seq_lens.  With an append, the
+    context includes the new token, and the call also reads k_new, v_new and
+    the two rotary table rows and writes the new key and value."""
+    if is_append(inp):
+        ctx = [int(x) + 1 for x in inp.cache_seqlens]
+    else:
+        ctx = [int(x) for x in inp.seq_lens]
     kv = sum(ctx) * inp.Hkv * inp.d * 2 * 2
     qo = 2 * inp.B * inp.Hq * inp.d * 2
     pages = sum((c + inp.page_size - 1) // inp.page_size for c in ctx)
-    return float(kv + qo + 4 * pages + 4 * inp.B)
+    extra = 0
+    if is_append(inp):
+        extra = 2 * (2 * inp.B * inp.Hkv * inp.d * 2)          # k_new, v_new read; k, v written
+        if inp.cos is not None:
+            extra += inp.B * 2 * (inp.rotary_dim // 2) * 4      # one cos and one sin row each
+    return float(kv + qo + 4 * pages + 4 * inp.B + extra)
 
 
 def load_peaks():
@@ -243,6 +257,16 @@ def oracle_decode_sample(din, n_req: int):
     """Times the fp64 oracle on the first n_req requests (all heads).
     Returns (algorithmic bytes of those requests, seconds)."""
     import oracle
+    if is_append(din):
+        sub = inputs.AppendInputs(**{**din.__dict__, "q": din.q[:n_req], "k_new": din.k_new[:n_req],
+                                     "v_new": din.v_new[:n_req],
+                                     "block_table": din.block_table[:n_req],
+                                     "cache_seqlens": din.cache_seqlens[:n_req]})
+        t0 = time.perf_counter()
+        oracle.decode_paged_append(sub.q, sub.k_new, sub.v_new, sub.k_pages, sub.v_pages,
+                                   sub.block_table, sub.cache_seqlens, sub.scale, sub.cos, sub.sin,
+                                   sub.rotary_dim or None, sub.interleaved)
+        return decode_bytes(sub), time.perf_counter() - t0
     sub = inputs.DecodeInputs("sample", din.q[:n_req], din.k_pages, din.v_pages,
                               din.block_table[:n_req], din.seq_lens[:n_req], din.page_size,
                               din.scale)
@@ -289,6 +313,7 @@ WORKLOAD_NAMES = {
     "window_prefill": inputs.WORKLOADS["window_prefill"],
     "softcap_prefill": inputs.WORKLOADS["softcap_prefill"],
     "alibi_prefill": inputs.WORKLOADS["alibi_prefill"],
+    "append_decode": inputs.WORKLOADS["append_decode"],
 }
 
 
@@ -304,6 +329,8 @@ def make_workload(name):
         din = inputs.long_decode()
     if name in ("window_prefill", "softcap_prefill", "alibi_prefill"):
         pin = getattr(inputs, name)()
+    if name == "append_decode":
+        din = inputs.append_decode()
     return pin, din
 
 
@@ -323,12 +350,19 @@ class DeviceWorkload:
                 self.variant["alibi_slopes"] = self.variant["alibi_slopes"].to(dev)
         if din is not None:
             self.dq, self.kp, self.vp = (t.to(dev) for t in (din.q, din.k_pages, din.v_pages))
-            self.bt, self.sl = din.block_table.to(dev), din.seq_lens.to(dev)
+            self.bt = din.block_table.to(dev)
+            self.sl = (din.cache_seqlens if is_append(din) else din.seq_lens).to(dev)
             # automatic page ranges (num_splits = 0); splits = the most ranges a
             # request can get, which sizes the workspace
             self.splits = api.decode_auto_splits(din.B, din.Hq, din.Hkv,
                                                  din.block_table.shape[1], din.page_size)
-            nbytes = api.decode_workspace_size(din.B, din.Hq, din.d, self.splits)
+            if is_append(din):
+                self.kn, self.vn = din.k_new.to(dev), din.v_new.to(dev)
+                self.cos = din.cos.to(dev) if din.cos is not None else None
+                self.sin = din.sin.to(dev) if din.sin is not None else None
+                nbytes = api.decode_append_workspace_size(din.B, din.Hq, din.d, self.splits)
+            else:
+                nbytes = api.decode_workspace_size(din.B, din.Hq, din.d, self.splits)
             self.ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) if nbytes else None
             self.do = torch.empty_like(self.dq)
             self.dlse = torch.empty(din.B, din.Hq, dtype=torch.float32, device=dev)
@@ -337,6 +371,7 @@ class DeviceWorkload:
         n = 1 if self.pin is not None else 0
         if self.din is not None:
             n += 1 + (2 if self.splits > 1 else 0)  # split kernel (+ plan and combine)
+            n += 1 if is_append(self.din) else 0    # append + RoPE kernel
         return n
 
     def prefill(self):
@@ -344,6 +379,13 @@ class DeviceWorkload:
                        self.pin.scale, self.max_len, **self.variant)
 
     def decode(self):
+        if is_append(self.din):
+            # the same slot is rewritten with the same values every call
+            api.fa_decode_paged_append(self.dq, self.kn, self.vn, self.kp, self.vp, self.bt,
+                                       self.sl, 0, self.do, self.dlse, self.din.scale, self.cos,
+                                       self.sin, self.din.rotary_dim or None,
+                                       self.din.interleaved, self.ws)
+            return
         api.fa_decode_paged(self.dq, self.kp, self.vp, self.bt, self.sl, 0, self.do,
                             self.dlse, self.din.scale, self.ws)
 
@@ -402,8 +444,14 @@ def time_e2e(w: DeviceWorkload, steps: int):
         host["lse"] = torch.empty(w.lse.shape, dtype=w.lse.dtype, pin_memory=True)
         d2h += w.o.numel() * 2 + w.lse.numel() * 4
     if din is not None:
-        for n, t in (("dq", din.q), ("kp", din.k_pages), ("vp", din.v_pages),
-                     ("bt", din.block_table), ("sl", din.seq_lens)):
+        srcs = [("dq", din.q), ("kp", din.k_pages), ("vp", din.v_pages),
+                ("bt", din.block_table),
+                ("sl", din.cache_seqlens if is_append(din) else din.seq_lens)]
+        if is_append(din):
+            srcs += [("kn", din.k_new), ("vn", din.v_new)]
+            if din.cos is not None:
+                srcs += [("cos", din.cos), ("sin", din.sin)]
+        for n, t in srcs:
             host[n] = t.pin_memory()
             h2d += t.numel() * t.element_size()
         host["do"] = torch.empty(w.do.shape, dtype=w.do.dtype, pin_memory=True)
@@ -428,6 +476,9 @@ def time_e2e(w: DeviceWorkload, steps: int):
             w.vp.copy_(host["vp"], non_blocking=True)
             w.bt.copy_(host["bt"], non_blocking=True)
             w.sl.copy_(host["sl"], non_blocking=True)
+            for n in ("kn", "vn", "cos", "sin"):
+                if n in host:
+                    getattr(w, n).copy_(host[n], non_blocking=True)
             w.decode()
             host["do"].copy_(w.do, non_blocking=True)
             host["dlse"].copy_(w.dlse, non_blocking=True)
@@ -493,7 +544,7 @@ def run_gpu(args, world, rank, local):
             "workspace_bytes": api.decode_workspace_size(din.B, din.Hq, din.d, w.splits),
             "roofline": roofline("decode", gbs / world, peaks["hbm_gbs"], "GB/s",
                                  dram_traffic("decode", din.name)),
-            "launches_per_call": 1 + (2 if w.splits > 1 else 0),
+            "launches_per_call": 1 + (2 if w.splits > 1 else 0) + (1 if is_append(din) else 0),
         }
     head = parts.get("prefill") or parts.get("decode")
     dominant = max(parts.values(), key=lambda p: p["ms"])

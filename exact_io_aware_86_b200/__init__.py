@@ -1,6 +1,6 @@
 """Exact IO-aware attention on B200 (sm_100a).
 
-Two entry points, both running entirely in this package's CUDA library
+Entry points, all running entirely in this package's CUDA library
 (``libfa.so``, C ABI declared in ``include/fa.h``):
 
 * ``prefill`` / ``fa_prefill``: causal or full attention over packed
@@ -8,19 +8,24 @@ Two entry points, both running entirely in this package's CUDA library
   an online softmax on the tcgen05 tensor cores.
 * ``decode_paged`` / ``fa_decode_paged``: one query token per request against
   a paged KV cache, split along the context and merged by log-sum-exp.
+* ``decode_paged_append`` / ``fa_decode_paged_append``: the same after
+  appending the new token's key and value to the cache, with optional RoPE.
 
 The Python layer only marshals arguments.  Importing the package loads
 nothing; the first call loads ``libfa.so`` and raises if it is missing.
 """
 from .api import (  # noqa: F401
     FAError,
+    decode_append_workspace_size,
     decode_auto_splits,
     decode_paged,
+    decode_paged_append,
     decode_paged_f32,
     decode_workspace_size,
     device_error,
     error_string,
     fa_decode_paged,
+    fa_decode_paged_append,
     fa_prefill,
     load_library,
     prefill,

@@ -49,6 +49,12 @@ def load_library(path: str = LIB_PATH):
     lib.fa_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32,
                                             i32, i32, i32, f32, vp]
     lib.fa_decode_paged_noalloc.restype = ctypes.c_int
+    lib.fa_decode_paged_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32,
+                                           i32, i32, i32, i32, f32, vp, vp, vp, i32, i32, i32, vp,
+                                           sz]
+    lib.fa_decode_paged_append.restype = ctypes.c_int
+    lib.fa_decode_append_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.fa_decode_append_workspace_size.restype = sz
     lib.fa_decode_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.fa_decode_workspace_size.restype = sz
     lib.fa_decode_auto_splits.argtypes = [i32, i32, i32, i32, i32, i32]
@@ -287,3 +293,65 @@ def device_error(stream=None) -> int:
     _check(load_library().fa_get_device_error(_stream(stream), ctypes.byref(code)),
            "fa_get_device_error")
     return code.value
+
+
+# --------------------------------------------------------------------------
+# decode with cache append (+ RoPE)
+# --------------------------------------------------------------------------
+def decode_append_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:
+    return int(load_library().fa_decode_append_workspace_size(B, Hq, d, num_splits))
+
+
+def fa_decode_paged_append(q, k_new, v_new, k_pages, v_pages, block_table, cache_seqlens,
+                           num_splits: int, o, lse=None, scale: float = 0.0, rotary_cos=None,
+                           rotary_sin=None, rotary_dim: int | None = None,
+                           rotary_interleaved: bool = False,
+                           workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Calls ``fa_decode_paged_append``: writes k_new/v_new (k rotated when
+    tables are given) into the page pool at cache_seqlens, then attends.
+    k_pages / v_pages are modified in place; cache_seqlens is not."""
+    B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
+        q, k_pages, v_pages, block_table, cache_seqlens, torch.bfloat16)
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n, torch.bfloat16, 3)
+        if tuple(t.shape) != (B, Hkv, d):
+            raise ValueError(f"{n} must be [B, Hkv, d]")
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    max_pos, rd = 0, 0
+    if (rotary_cos is None) != (rotary_sin is None):
+        raise ValueError("give both rotary_cos and rotary_sin, or neither")
+    if rotary_cos is not None:
+        _need(rotary_cos, "rotary_cos", torch.float32, 2)
+        _need(rotary_sin, "rotary_sin", torch.float32, 2)
+        if rotary_sin.shape != rotary_cos.shape:
+            raise ValueError("rotary_cos and rotary_sin shapes differ")
+        max_pos = rotary_cos.shape[0]
+        rd = int(rotary_dim) if rotary_dim is not None else 2 * rotary_cos.shape[1]
+        if rotary_cos.shape[1] != rd // 2:
+            raise ValueError("rotary tables need rotary_dim / 2 columns")
+    ws_bytes = 0
+    if workspace is not None:
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load_library().fa_decode_paged_append(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+        _ptr(cache_seqlens), page_size, int(num_splits), _ptr(o), _stream(stream), B, Hq, Hkv, d,
+        max_blocks, num_pages, float(scale), _ptr(lse), _ptr(rotary_cos), _ptr(rotary_sin),
+        max_pos, rd, int(bool(rotary_interleaved)), _ptr(workspace), ws_bytes),
+        "fa_decode_paged_append")
+
+
+def decode_paged_append(q, k_new, v_new, k_pages, v_pages, block_table, cache_seqlens,
+                        num_splits: int = 0, scale: float = 0.0, rotary_cos=None, rotary_sin=None,
+                        rotary_dim: int | None = None, rotary_interleaved: bool = False,
+                        return_lse: bool = True, stream=None):
+    """Allocates O (and LSE) and runs ``fa_decode_paged_append``.  Returns (o, lse or None)."""
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if return_lse else None
+    fa_decode_paged_append(q, k_new, v_new, k_pages, v_pages, block_table, cache_seqlens,
+                           num_splits, o, lse, scale, rotary_cos, rotary_sin, rotary_dim,
+                           rotary_interleaved, None, stream)
+    return o, lse

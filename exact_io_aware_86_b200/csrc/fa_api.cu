@@ -17,6 +17,7 @@
 #include "prefill_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "debug_f32.cuh"
+#include "append_rope.cuh"
 
 namespace {
 
@@ -386,6 +387,98 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
   else
     st = launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, page_size, num_splits, o,
                             s, B, Hq, Hkv, max_blocks_per_seq, num_pages, scale, lse, ws);
+  if (owned && cudaFreeAsync(ws, s) != cudaSuccess && st == FA_OK) st = FA_ERR_CUDA;
+  return st;
+}
+
+size_t fa_decode_append_workspace_size(int B, int Hq, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || d <= 0) return 0;
+  return round_up((size_t)B * Hq * d * 2, 256) + round_up((size_t)B * 4, 256) +
+         fa_decode_workspace_size(B, Hq, d, num_splits);
+}
+
+fa_status fa_decode_paged_append(const void* q, const void* k_new, const void* v_new,
+                                 void* k_pages, void* v_pages, const int32_t* block_table,
+                                 const int32_t* cache_seqlens, int page_size, int num_splits,
+                                 void* o, fa_stream_t stream, int B, int Hq, int Hkv, int d,
+                                 int max_blocks_per_seq, int num_pages, float scale, float* lse,
+                                 const float* rotary_cos, const float* rotary_sin,
+                                 int rotary_max_pos, int rotary_dim, int rotary_interleaved,
+                                 void* workspace, size_t workspace_bytes) {
+  if (!q || !k_new || !v_new || !k_pages || !v_pages || !block_table || !cache_seqlens || !o)
+    return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || page_size < 1 || num_splits < 0 ||
+      max_blocks_per_seq < 1 || num_pages < 0)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pages, 16) ||
+      !aligned(v_pages, 16) || !aligned(o, 16) || !aligned(block_table, 4) ||
+      !aligned(cache_seqlens, 4) || (lse && !aligned(lse, 4)) ||
+      (workspace && !aligned(workspace, 256)))
+    return FA_ERR_INVALID_ARG;
+  if ((rotary_cos == nullptr) != (rotary_sin == nullptr)) return FA_ERR_INVALID_ARG;
+  if (rotary_cos && (rotary_dim < 2 || rotary_dim > d || rotary_dim % 2 != 0 ||
+                     rotary_max_pos < 1 || !aligned(rotary_cos, 4) || !aligned(rotary_sin, 4)))
+    return FA_ERR_INVALID_ARG;
+  // the attention step has the limits of fa_decode_paged
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > fa::decode::MAX_GROUP) return FA_ERR_UNSUPPORTED;
+  if (page_size % fa::decode::TOK != 0) return FA_ERR_UNSUPPORTED;
+  if ((long long)num_pages * page_size > 0x7fffffffLL ||
+      (long long)max_blocks_per_seq * page_size > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv / heads_per_cta(Hkv) > 65535) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  const int S = num_splits == 0
+                    ? fa_decode_auto_splits(B, Hq, Hkv, max_blocks_per_seq, page_size, 0)
+                    : num_splits;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t q_bytes = round_up((size_t)B * Hq * d * 2, 256);
+  const size_t l_bytes = round_up((size_t)B * 4, 256);
+  const size_t need = fa_decode_append_workspace_size(B, Hq, d, S);
+  void* ws = workspace;
+  bool owned = false;
+  if (ws) {
+    if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+  } else {
+    if (cudaMallocAsync(&ws, need, s) != cudaSuccess) return FA_ERR_CUDA;
+    owned = true;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  fa::append::Params ap;
+  ap.q = static_cast<const __nv_bfloat16*>(q);
+  ap.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  ap.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  ap.k_pages = static_cast<__nv_bfloat16*>(k_pages);
+  ap.v_pages = static_cast<__nv_bfloat16*>(v_pages);
+  ap.block_table = block_table;
+  ap.cache_seqlens = cache_seqlens;
+  ap.cos = rotary_cos;
+  ap.sin = rotary_sin;
+  ap.q_rot = reinterpret_cast<__nv_bfloat16*>(w);
+  ap.seq_lens_new = reinterpret_cast<int32_t*>(w + q_bytes);
+  ap.B = B;
+  ap.Hq = Hq;
+  ap.Hkv = Hkv;
+  ap.d = d;
+  ap.page_size = page_size;
+  ap.max_blocks = max_blocks_per_seq;
+  ap.num_pages = num_pages;
+  ap.max_pos = rotary_cos ? rotary_max_pos : 0;
+  ap.rd = rotary_cos ? rotary_dim : 0;
+  ap.interleaved = rotary_interleaved ? 1 : 0;
+  fa::append::append_rope_kernel<<<B, fa::append::THREADS, 0, s>>>(ap);
+  fa_status st = cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (st == FA_OK) {
+    void* dws = (need > q_bytes + l_bytes) ? static_cast<void*>(w + q_bytes + l_bytes) : nullptr;
+    if (d == 64)
+      st = launch_decode<64>(ap.q_rot, k_pages, v_pages, block_table, ap.seq_lens_new, page_size,
+                             num_splits, o, s, B, Hq, Hkv, max_blocks_per_seq, num_pages, scale,
+                             lse, dws);
+    else
+      st = launch_decode<128>(ap.q_rot, k_pages, v_pages, block_table, ap.seq_lens_new,
+                              page_size, num_splits, o, s, B, Hq, Hkv, max_blocks_per_seq,
+                              num_pages, scale, lse, dws);
+  }
   if (owned && cudaFreeAsync(ws, s) != cudaSuccess && st == FA_OK) st = FA_ERR_CUDA;
   return st;
 }

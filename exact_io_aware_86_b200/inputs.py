@@ -207,6 +207,9 @@ WORKLOADS = {
                       "Hq=32 Hkv=8 d=128",
     "softcap_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 with softcap 50",
     "alibi_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 with ALiBi slopes",
+    # inference KV cache step (skill page section 3.5)
+    "append_decode": "paged decode with cache append + RoPE (rotary_dim 128), 64 requests, "
+                     "Hq=32 Hkv=8 d=128, ctx~U[1024,32767], page 16",
 }
 
 
@@ -264,6 +267,84 @@ def alibi_prefill() -> PrefillInputs:
     inp.name = "alibi_prefill"
     inp.meta["variant"] = {"alibi_slopes": alibi_slopes_geometric(16)}
     return inp
+
+
+@dataclass
+class AppendInputs:
+    """One decode step that appends a token per request (skill page 3.5)."""
+    name: str
+    q: torch.Tensor              # [B, Hq, d] bf16
+    k_new: torch.Tensor          # [B, Hkv, d] bf16
+    v_new: torch.Tensor
+    k_pages: torch.Tensor        # [num_pages, page_size, Hkv, d] bf16 (room for ctx + 1)
+    v_pages: torch.Tensor
+    block_table: torch.Tensor    # [B, max_blocks] int32
+    cache_seqlens: torch.Tensor  # [B] int32: tokens already cached
+    page_size: int
+    scale: float
+    cos: torch.Tensor | None     # [max_pos, rotary_dim / 2] fp32
+    sin: torch.Tensor | None
+    rotary_dim: int
+    interleaved: bool
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def B(self):
+        return self.q.shape[0]
+
+    @property
+    def Hq(self):
+        return self.q.shape[1]
+
+    @property
+    def Hkv(self):
+        return self.k_pages.shape[2]
+
+    @property
+    def d(self):
+        return self.q.shape[2]
+
+
+def rope_tables(max_pos: int, rotary_dim: int, base: float = 10000.0):
+    """fp32 cos/sin tables [max_pos, rotary_dim/2] of the angles
+    pos * base^(-2i/rotary_dim), the usual RoPE frequencies (computed in
+    fp64, rounded once).  Input data: the pages give the argument, not its
+    values."""
+    half = rotary_dim // 2
+    pos = torch.arange(max_pos, dtype=torch.float64).unsqueeze(1)
+    inv = base ** (-2.0 * torch.arange(half, dtype=torch.float64) / rotary_dim)
+    ang = pos * inv
+    return torch.cos(ang).float().contiguous(), torch.sin(ang).float().contiguous()
+
+
+def make_append_decode(ctx, Hq: int, Hkv: int, d: int, page_size: int, seed: int,
+                       rotary_dim: int = 0, interleaved: bool = False, max_pos: int | None = None,
+                       name: str = "append_decode") -> AppendInputs:
+    """Paged cache holding ctx[b] tokens of request b, with room for one more
+    (pages placed by a seeded permutation), plus the new token's q/k/v."""
+    gen = torch.Generator().manual_seed(seed)
+    bt, num_pages = paged_layout([int(c) + 1 for c in ctx], page_size, gen)
+    B = len(ctx)
+    q = randn_bf16((B, Hq, d), gen)
+    k_new = randn_bf16((B, Hkv, d), gen)
+    v_new = randn_bf16((B, Hkv, d), gen)
+    k = randn_bf16((num_pages, page_size, Hkv, d), gen)
+    v = randn_bf16((num_pages, page_size, Hkv, d), gen)
+    cos = sin = None
+    if rotary_dim:
+        cos, sin = rope_tables(max_pos if max_pos is not None else max(ctx) + 1, rotary_dim)
+    return AppendInputs(name=name, q=q, k_new=k_new, v_new=v_new, k_pages=k, v_pages=v,
+                        block_table=bt, cache_seqlens=torch.tensor([int(c) for c in ctx], dtype=torch.int32),
+                        page_size=page_size, scale=fp32_scale(d), cos=cos, sin=sin,
+                        rotary_dim=rotary_dim, interleaved=interleaved, meta={"seed": seed})
+
+
+def append_decode() -> AppendInputs:
+    """The paged-decode workload's shape, one token appended per request, with
+    RoPE over the full head dimension."""
+    gen = torch.Generator().manual_seed(1007)
+    ctx = uniform_lengths(64, 1024, 32767, gen)
+    return make_append_decode(ctx, 32, 8, 128, 16, seed=1007, rotary_dim=128, max_pos=32768)
 
 
 def _decode_from_lengths(name, seq_lens, page_size, seed, gen):

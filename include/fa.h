@@ -172,6 +172,51 @@ fa_status fa_decode_paged_noalloc(const void *q, const void *k_pages, const void
                                   int B, int Hq, int Hkv, int d, int max_blocks_per_seq,
                                   int num_pages, float scale, float *lse);
 
+/*
+ * Decode step that first appends the new token to the cache ("flash-attention"
+ * skill page, section 3.5: flash_attn_with_kvcache with k_new, v_new,
+ * cache_seqlens, block_table and on-the-fly rotary embedding).
+ *
+ *   q             bf16 [B, Hq, d]    the new token's queries (not modified)
+ *   k_new, v_new  bf16 [B, Hkv, d]   its key and value
+ *   k_pages,      bf16 [num_pages, page_size, Hkv, d]   the page pool,
+ *   v_pages       MODIFIED: the new key and value are written at position
+ *                 pos = cache_seqlens[b] of request b, i.e. page
+ *                 block_table[b][pos / page_size], slot pos % page_size
+ *   cache_seqlens int32 [B], device: tokens already cached per request
+ *                 (not modified; the caller advances it)
+ *   rotary_cos,   fp32 [rotary_max_pos, rotary_dim / 2], device, or both NULL
+ *   rotary_sin    (no rotation).  With tables, q and k_new are rotated at pos:
+ *                 pair i is (x_i, x_{i + rotary_dim/2}), or (x_{2i}, x_{2i+1})
+ *                 when rotary_interleaved != 0, turned by the angle with
+ *                 cosine cos[pos][i] and sine sin[pos][i]; dimensions at or
+ *                 past rotary_dim are unchanged.  The rotation is computed in
+ *                 fp64 and rounded once to bf16 (nearest, ties to even).
+ *                 rotary_dim must be even, 2 <= rotary_dim <= d.
+ *   workspace     >= fa_decode_append_workspace_size(B, Hq, d, resolved
+ *                 num_splits) bytes, 256-byte aligned, or NULL (allocated
+ *                 stream-ordered)
+ * Every query then attends to the pos + 1 tokens of its request, exactly as
+ * fa_decode_paged with seq_lens = cache_seqlens + 1; the other arguments and
+ * limits are those of fa_decode_paged.  Requests must append to distinct
+ * page slots.  A position outside the block table or the rotary table, or an
+ * unused page there, records FA_ERR_DEVICE_BOUNDS; that request writes
+ * nothing to the cache and yields O = 0, LSE = -inf.
+ */
+fa_status fa_decode_paged_append(const void *q, const void *k_new, const void *v_new,
+                                 void *k_pages, void *v_pages, const int32_t *block_table,
+                                 const int32_t *cache_seqlens, int page_size, int num_splits,
+                                 void *o, fa_stream_t stream, int B, int Hq, int Hkv, int d,
+                                 int max_blocks_per_seq, int num_pages, float scale, float *lse,
+                                 const float *rotary_cos, const float *rotary_sin,
+                                 int rotary_max_pos, int rotary_dim, int rotary_interleaved,
+                                 void *workspace, size_t workspace_bytes);
+
+/* Workspace of fa_decode_paged_append: the rotated queries (bf16
+ * [B, Hq, d]), the new context lengths (int32 [B]) and the split workspace
+ * of fa_decode_workspace_size, each rounded up to 256 bytes. */
+size_t fa_decode_append_workspace_size(int B, int Hq, int d, int num_splits);
+
 /* Bytes of workspace fa_decode_paged needs for this shape and split count
  * (partial outputs fp32 [B, Hq, S, d], partial LSEs fp32 [B, Hq, S] and
  * the per-request range counts int32 [B+1]); 0 when S <= 1. */

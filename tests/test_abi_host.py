@@ -30,7 +30,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("fa_prefill", "fa_prefill_ex", "fa_decode_paged", "fa_decode_workspace_size",
+    for n in ("fa_prefill", "fa_prefill_ex", "fa_decode_paged", "fa_decode_paged_append",
+              "fa_decode_append_workspace_size", "fa_decode_workspace_size",
               "fa_decode_auto_splits", "fa_get_error_string", "fa_get_device_error"):
         assert n in names
 
@@ -117,6 +118,32 @@ def test_decode_argument_checks(lib):
     need = lib.fa_decode_workspace_size(2, 32, 128, 4)
     assert _decode(lib, S=4, ws=ctypes.c_void_p(0x10000), wsb=need - 1) == api.FA_ERR_INVALID_ARG
     assert _decode(lib, B=0) == api.FA_OK
+
+
+def _append(lib, **kw):
+    a = dict(q=FAKE, kn=FAKE, vn=FAKE, k=FAKE, v=FAKE, bt=FAKE, cs=FAKE, ps=16, S=0, o=FAKE,
+             stream=None, B=2, Hq=32, Hkv=8, d=128, maxb=4, npages=8, scale=0.0, lse=None,
+             cos=None, sin=None, maxpos=0, rd=0, inter=0, ws=None, wsb=0)
+    a.update(kw)
+    return lib.fa_decode_paged_append(a["q"], a["kn"], a["vn"], a["k"], a["v"], a["bt"], a["cs"],
+                                      a["ps"], a["S"], a["o"], a["stream"], a["B"], a["Hq"],
+                                      a["Hkv"], a["d"], a["maxb"], a["npages"], a["scale"],
+                                      a["lse"], a["cos"], a["sin"], a["maxpos"], a["rd"],
+                                      a["inter"], a["ws"], a["wsb"])
+
+
+def test_decode_append_argument_checks(lib):
+    assert _append(lib, kn=None) == api.FA_ERR_INVALID_ARG
+    assert _append(lib, cos=FAKE) == api.FA_ERR_INVALID_ARG                    # cos without sin
+    assert _append(lib, cos=FAKE, sin=FAKE, maxpos=10, rd=3) == api.FA_ERR_INVALID_ARG   # odd
+    assert _append(lib, cos=FAKE, sin=FAKE, maxpos=10, rd=130) == api.FA_ERR_INVALID_ARG  # > d
+    assert _append(lib, cos=FAKE, sin=FAKE, maxpos=0, rd=64) == api.FA_ERR_INVALID_ARG
+    assert _append(lib, d=96) == api.FA_ERR_UNSUPPORTED
+    assert _append(lib, ps=8) == api.FA_ERR_UNSUPPORTED
+    need = lib.fa_decode_append_workspace_size(2, 32, 128, 4)
+    assert need == (lib.fa_decode_workspace_size(2, 32, 128, 4) + 2 * 32 * 128 * 2 + 256)
+    assert _append(lib, S=4, ws=ctypes.c_void_p(0x10000), wsb=need - 1) == api.FA_ERR_INVALID_ARG
+    assert _append(lib, B=0) == api.FA_OK
 
 
 def test_decode_workspace_is_linear_in_splits_not_context(lib):
