@@ -108,6 +108,10 @@ class Oracle:
         lib.oracle_rope.argtypes = [vp, ci, c64, ci, vp, vp, vp, c64, ci, ci, vp]
         lib.oracle_decode_paged_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci,
                                                    ci, c64, cd, vp, vp, c64, ci, ci, vp, vp, vp]
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_prefill_fp8.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, cd, cd, cd, cd, vp, vp]
+        lib.oracle_prefill_fp8.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_set_num_threads.argtypes = [ci]
         for f in (lib.oracle_prefill_rows_ex, lib.oracle_prefill_ex, lib.oracle_prefill_probs,
@@ -281,6 +285,38 @@ class Oracle:
         return o, lse, kp, vpg, qr
 
 
+    def e4m3_value(self, byte: int) -> float:
+        """Exact value of one e4m3 byte."""
+        return float(self._lib.oracle_e4m3_value(int(byte) & 0xFF))
+
+    def prefill_fp8(self, q, k, v, cu_seqlens, causal: bool, scale: float, q_descale: float = 1.0,
+                    k_descale: float = 1.0, v_descale: float = 1.0):
+        """Exact attention of e4m3 inputs (torch float8_e4m3fn tensors, or uint8
+        bytes) times their per-tensor descale factors.  Returns (o, lse) as
+        in ``prefill``."""
+        def raw(x):
+            import torch
+            if isinstance(x, torch.Tensor):
+                x = x.detach().cpu().contiguous()
+                if x.dtype != torch.uint8:
+                    x = x.view(torch.uint8)
+                return x.numpy()
+            return np.ascontiguousarray(x, dtype=np.uint8)
+        qa, ka, va = raw(q), raw(k), raw(v)
+        cu = _int_np(cu_seqlens, np.int32)
+        T, Hq, d = qa.shape
+        Hkv = ka.shape[1]
+        B = cu.shape[0] - 1
+        o = np.zeros((T, Hq, d), np.float64)
+        lse = np.zeros((Hq, T), np.float64)
+        rc = self._lib.oracle_prefill_fp8(_ptr(qa), _ptr(ka), _ptr(va), _ptr(cu), B, Hq, Hkv, d,
+                                          int(bool(causal)), float(scale), float(q_descale),
+                                          float(k_descale), float(v_descale), _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError(f"oracle_prefill_fp8 rejected its arguments (rc={rc})")
+        return o, lse
+
+
 _default: Oracle | None = None
 
 
@@ -319,6 +355,14 @@ def rope(*args, **kw):
 
 def decode_paged_append(*args, **kw):
     return default().decode_paged_append(*args, **kw)
+
+
+def e4m3_value(*args, **kw):
+    return default().e4m3_value(*args, **kw)
+
+
+def prefill_fp8(*args, **kw):
+    return default().prefill_fp8(*args, **kw)
 
 
 def set_num_threads(n: int) -> None:

@@ -45,6 +45,10 @@
  *    bf16, so the rotated key is the exact rotation rounded once to bf16
  *    (nearest, ties to even), and the rotated query likewise (it feeds a
  *    bf16 product).
+ *  - FP8 (skill page, comparison tables: FA3/FA4 support FP8): Q, K and V
+ *    stored as OCP e4m3 bytes (4 exponent bits, bias 7, 3 mantissa bits, no
+ *    infinities) with one descale factor per tensor; the attention is the
+ *    plain definition on the exact values descale * e4m3.
  *
  * Precision: every product and sum is in double.  Inputs are read in the
  * caller's element type (bf16 bit patterns, fp32 or fp64) and upcast
@@ -663,6 +667,57 @@ int oracle_decode_paged_append(const uint16_t *q, const uint16_t *k_new, const u
     free(tmp);
     free(rot);
     return bad ? -1 : 0;
+}
+
+/* Exact value of an OCP e4m3 byte: sign, 4-bit exponent (bias 7), 3-bit
+ * mantissa; exponent 0 is subnormal (m/8 * 2^-6); 0x7F/0xFF are NaN. */
+double oracle_e4m3_value(uint8_t b)
+{
+    int sign = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/*
+ * FP8 prefill: q [T, Hq, d], k, v [T, Hkv, d] as e4m3 bytes with per-tensor
+ * descale factors; the attention of the exact values descale * e4m3 (fp64),
+ * with the masks of oracle_prefill.  o [T, Hq, d] double, lse [Hq, T].
+ */
+int oracle_prefill_fp8(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                       const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                       double scale, double q_descale, double k_descale, double v_descale,
+                       double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || d <= 0)
+        return -1;
+    size_t T = (size_t)cu_seqlens[B];
+    size_t nq = T * (size_t)Hq * (size_t)d, nk = T * (size_t)Hkv * (size_t)d;
+    double *qd = (double *)malloc((nq ? nq : 1) * sizeof(double));
+    double *kd = (double *)malloc((nk ? nk : 1) * sizeof(double));
+    double *vd = (double *)malloc((nk ? nk : 1) * sizeof(double));
+    if (!qd || !kd || !vd) {
+        free(qd);
+        free(kd);
+        free(vd);
+        return -1;
+    }
+    for (size_t i = 0; i < nq; ++i)
+        qd[i] = q_descale * oracle_e4m3_value(q[i]);
+    for (size_t i = 0; i < nk; ++i) {
+        kd[i] = k_descale * oracle_e4m3_value(k[i]);
+        vd[i] = v_descale * oracle_e4m3_value(v[i]);
+    }
+    int rc = oracle_prefill(qd, kd, vd, OR_F64, cu_seqlens, B, Hq, Hkv, d, causal, scale, o, lse);
+    free(qd);
+    free(kd);
+    free(vd);
+    return rc;
 }
 
 /* Threads the OpenMP runtime will use (for reporting). */

@@ -18,7 +18,8 @@ from oracle import build as oracle_build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_variant_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_append_pins.py")]
+        os.path.join(ROOT, "tests", "test_oracle_append_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_fp8_pins.py")]
 
 MUTANTS = {
     "scale_dropped": ("s[j] = scale * dot;", "s[j] = dot;"),
@@ -71,6 +72,12 @@ MUTANTS = {
     "value_rotated_like_key": ("v_pages[dst + (size_t)c] = v_new[src + (size_t)c];",
                                "v_pages[dst + (size_t)c] = bf16_bits(round_bf16(rot[c]));"),
     "bf16_rounding_truncates": ("double r = nearbyint(scaled);", "double r = trunc(scaled);"),
+    # FP8 inputs
+    "e4m3_bias_off_by_one": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_subnormal_scale": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
+    "e4m3_mantissa_width": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 16.0, e - 7);"),
+    "fp8_value_descale_dropped": ("vd[i] = v_descale * oracle_e4m3_value(v[i]);", "vd[i] = oracle_e4m3_value(v[i]);"),
+    "fp8_key_descale_on_query": ("kd[i] = k_descale * oracle_e4m3_value(k[i]);", "kd[i] = q_descale * oracle_e4m3_value(k[i]);"),
 }
 
 
