@@ -111,6 +111,10 @@ def variant_of(pin) -> dict:
     return dict(pin.meta.get("variant", {})) if pin is not None else {}
 
 
+def is_fp8(pin) -> bool:
+    return pin is not None and pin.q.dtype == torch.float8_e4m3fn
+
+
 def is_append(inp) -> bool:
     return isinstance(inp, inputs.AppendInputs)
 
@@ -247,8 +251,13 @@ def oracle_prefill_sample(pin, n_pairs: int):
         rt.extend(range(start, start + L))
         rh.extend([h] * L)
         flops += prefill_flops([L], 1, pin.d, pin.causal, var.get("window", (-1, -1)))
+    q, k, v = pin.q, pin.k, pin.v
+    if q.dtype == torch.float8_e4m3fn:
+        # the oracle's e4m3 path is decode-then-fp64; decode once, outside the timing
+        qs, ks, vs = pin.meta["descale"]
+        q, k, v = q.double() * qs, k.double() * ks, v.double() * vs
     t0 = time.perf_counter()
-    oracle.prefill_rows(pin.q, pin.k, pin.v, pin.cu_seqlens, pin.causal, pin.scale,
+    oracle.prefill_rows(q, k, v, pin.cu_seqlens, pin.causal, pin.scale,
                         np.array(rt), np.array(rh), **var)
     return flops, time.perf_counter() - t0
 
@@ -314,6 +323,7 @@ WORKLOAD_NAMES = {
     "softcap_prefill": inputs.WORKLOADS["softcap_prefill"],
     "alibi_prefill": inputs.WORKLOADS["alibi_prefill"],
     "append_decode": inputs.WORKLOADS["append_decode"],
+    "fp8_prefill": inputs.WORKLOADS["fp8_prefill"],
 }
 
 
@@ -327,7 +337,7 @@ def make_workload(name):
         din = inputs.paged_decode()
     if name == "long_decode":
         din = inputs.long_decode()
-    if name in ("window_prefill", "softcap_prefill", "alibi_prefill"):
+    if name in ("window_prefill", "softcap_prefill", "alibi_prefill", "fp8_prefill"):
         pin = getattr(inputs, name)()
     if name == "append_decode":
         din = inputs.append_decode()
@@ -342,7 +352,7 @@ class DeviceWorkload:
         if pin is not None:
             self.q, self.k, self.v = (t.to(dev) for t in (pin.q, pin.k, pin.v))
             self.cu = pin.cu_seqlens.to(dev)
-            self.o = torch.empty_like(self.q)
+            self.o = torch.empty(self.q.shape, dtype=torch.bfloat16, device=dev)
             self.lse = torch.empty(pin.Hq, pin.T, dtype=torch.float32, device=dev)
             self.max_len = max(pin.lengths)
             self.variant = variant_of(pin)
@@ -375,6 +385,11 @@ class DeviceWorkload:
         return n
 
     def prefill(self):
+        if self.pin.q.dtype == torch.float8_e4m3fn:
+            qs, ks, vs = self.pin.meta["descale"]
+            api.fa_prefill_fp8(self.q, self.k, self.v, self.o, self.lse, self.cu, self.pin.causal,
+                               self.pin.scale, qs, ks, vs, self.max_len)
+            return
         api.fa_prefill(self.q, self.k, self.v, self.o, self.lse, self.cu, self.pin.causal,
                        self.pin.scale, self.max_len, **self.variant)
 
@@ -530,7 +545,10 @@ def run_gpu(args, world, rank, local):
         parts["prefill"] = {
             "workload": pin.name, "value": round(tf, 2), "unit": "TFLOP/s",
             "ms": round(pre_ms, 4), "ms_min": round(min(pre), 4), "flops": fl,
-            "roofline": roofline("prefill", tf / world, peaks["bf16_tflops"], "TFLOP/s",
+            # an e4m3 contraction takes the fp8 peak: the measured bf16 peak times
+            # the nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
+            "roofline": roofline("prefill", tf / world,
+                                 peaks["bf16_tflops"] * (2.0 if is_fp8(pin) else 1.0), "TFLOP/s",
                                  dram_traffic("prefill", pin.name)),
             "launches_per_call": 1,
         }
@@ -570,7 +588,7 @@ def run_gpu(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "e4m3" if is_fp8(pin) else "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD_NAMES[args.workload],
                    "l2": "256 MB buffer written between steps; decode KV (4.4 GB) exceeds L2",

@@ -8,6 +8,8 @@ Entry points, all running entirely in this package's CUDA library
   an online softmax on the tcgen05 tensor cores.
 * ``decode_paged`` / ``fa_decode_paged``: one query token per request against
   a paged KV cache, split along the context and merged by log-sum-exp.
+* ``prefill_fp8`` / ``fa_prefill_fp8``: the prefill on e4m3 inputs with
+  descale factors, both products in FP8 on the tensor cores.
 * ``decode_paged_append`` / ``fa_decode_paged_append``: the same after
   appending the new token's key and value to the cache, with optional RoPE.
 
@@ -27,7 +29,9 @@ from .api import (  # noqa: F401
     fa_decode_paged,
     fa_decode_paged_append,
     fa_prefill,
+    fa_prefill_fp8,
     load_library,
     prefill,
     prefill_f32,
+    prefill_fp8,
 )

@@ -44,6 +44,9 @@ def load_library(path: str = LIB_PATH):
     vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, i32]
     lib.fa_prefill_ex.argtypes = lib.fa_prefill.argtypes + [i32, i32, f32, vp, i32]
+    lib.fa_prefill_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32,
+                                   f32, vp, i32, i32]
+    lib.fa_prefill_fp8.restype = ctypes.c_int
     lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32, i32, i32,
                                     i32, f32, vp, vp, sz]
     lib.fa_decode_paged_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i32, i32,
@@ -172,6 +175,42 @@ def prefill(q, k, v, cu_seqlens, causal: bool = True, scale: float = 0.0,
     lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device) if return_lse else None
     fa_prefill(q, k, v, o, lse, cu_seqlens, causal, scale, max_seqlen, stream, window=window,
                softcap=softcap, alibi_slopes=alibi_slopes)
+    return o, lse
+
+
+def fa_prefill_fp8(q, k, v, o, lse, cu_seqlens, causal: bool, scale: float = 0.0,
+                   q_descale: float = 1.0, k_descale: float = 1.0, v_descale: float = 1.0,
+                   max_seqlen: int | None = None, stream=None) -> None:
+    """Calls ``fa_prefill_fp8``: q [T, Hq, 128], k/v [T, Hkv, 128] as
+    torch.float8_e4m3fn, o bf16 [T, Hq, 128], lse fp32 [Hq, T] or None."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.float8_e4m3fn, 3)
+    _need(o, "o", torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (T, Hkv, d) or v.shape != k.shape or o.shape != q.shape:
+        raise ValueError("q/k/v/o shapes disagree")
+    if lse is not None and lse.shape != (Hq, T):
+        raise ValueError("lse must be [Hq, T]")
+    B = cu_seqlens.numel() - 1
+    ms = T if max_seqlen is None else int(max_seqlen)
+    _check(load_library().fa_prefill_fp8(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), B, Hq, Hkv, d,
+        int(bool(causal)), float(scale), float(q_descale), float(k_descale), float(v_descale),
+        _stream(stream), T, ms), "fa_prefill_fp8")
+
+
+def prefill_fp8(q, k, v, cu_seqlens, causal: bool = True, scale: float = 0.0,
+                q_descale: float = 1.0, k_descale: float = 1.0, v_descale: float = 1.0,
+                max_seqlen: int | None = None, return_lse: bool = True, stream=None):
+    """Allocates O (bf16) and LSE and runs ``fa_prefill_fp8``.  Returns (o, lse or None)."""
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(q.shape[1], q.shape[0], dtype=torch.float32, device=q.device) if return_lse else None
+    fa_prefill_fp8(q, k, v, o, lse, cu_seqlens, causal, scale, q_descale, k_descale, v_descale,
+                   max_seqlen, stream)
     return o, lse
 
 

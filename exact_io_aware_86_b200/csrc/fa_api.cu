@@ -47,14 +47,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle; dims/strides innermost first,
-// strides in bytes for dims 1.. (dim 0 is contiguous).
+// Tensor map with 128-byte swizzle (bf16 elements, or bytes for e4m3);
+// dims/strides innermost first, strides in bytes for dims 1.. (dim 0 is
+// contiguous).
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides, const cuuint32_t* box) {
+              const cuuint64_t* strides, const cuuint32_t* box, bool bytes = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+  const CUresult r = fn(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        (cuuint32_t)rank,
                         const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -98,23 +100,25 @@ struct Variant {
   bool general() const { return softcap > 0.f || alibi != nullptr || wl >= 0 || wr > 0; }
 };
 
-template <int D, bool GENERAL>
+template <int D, bool GENERAL, bool FP8 = false>
 fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                          const int32_t* cu, int B, int Hq, int Hkv, int causal, float scale,
-                         cudaStream_t stream, int T, int max_seqlen, const Variant& var) {
+                         cudaStream_t stream, int T, int max_seqlen, const Variant& var,
+                         float qk_descale = 1.f, float v_descale = 1.f) {
   using namespace fa::prefill;
+  using C = Cfg<D, FP8>;
   CUtensorMap tq, tk, tv;
-  const cuuint32_t box[2] = {64, (cuuint32_t)BM};
+  const cuuint32_t box[2] = {(cuuint32_t)C::PANEL_ELEMS, (cuuint32_t)BM};  // 128 B x 128 rows
   {
     const cuuint64_t dims[2] = {(cuuint64_t)Hq * D, (cuuint64_t)T};
-    const cuuint64_t str[1] = {(cuuint64_t)Hq * D * 2};
-    if (!make_map(&tq, q, 2, dims, str, box)) return FA_ERR_CUDA;
+    const cuuint64_t str[1] = {(cuuint64_t)Hq * D * C::ESIZE};
+    if (!make_map(&tq, q, 2, dims, str, box, FP8)) return FA_ERR_CUDA;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)Hkv * D, (cuuint64_t)T};
-    const cuuint64_t str[1] = {(cuuint64_t)Hkv * D * 2};
-    if (!make_map(&tk, k, 2, dims, str, box)) return FA_ERR_CUDA;
-    if (!make_map(&tv, v, 2, dims, str, box)) return FA_ERR_CUDA;
+    const cuuint64_t str[1] = {(cuuint64_t)Hkv * D * C::ESIZE};
+    if (!make_map(&tk, k, 2, dims, str, box, FP8)) return FA_ERR_CUDA;
+    if (!make_map(&tv, v, 2, dims, str, box, FP8)) return FA_ERR_CUDA;
   }
   Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -126,7 +130,8 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   p.group = Hq / Hkv;
   p.T = T;
   p.causal = causal ? 1 : 0;
-  p.scale_log2 = resolve_scale(scale, D) * kLog2e;
+  p.scale_log2 = resolve_scale(scale, D) * qk_descale * kLog2e;
+  p.o_scale = v_descale;
   p.num_levels = (max_seqlen + ROWS_PER_ITEM - 1) / ROWS_PER_ITEM;
   p.wl = var.wl;
   p.wr = var.wr;
@@ -143,18 +148,18 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   if ((upper + grid - 1) / grid > MAX_ITEMS_PER_CTA) grid = (upper + MAX_ITEMS_PER_CTA - 1) / MAX_ITEMS_PER_CTA;
   if (grid > 0x7fffffff) return FA_ERR_UNSUPPORTED;
 
-  const int smem = smem_bytes<D>();
-  static bool attr_ok = set_smem(prefill_kernel<D, GENERAL>, smem);
+  const int smem = smem_bytes<D, FP8>();
+  static bool attr_ok = set_smem(prefill_kernel<D, GENERAL, FP8>, smem);
   if (!attr_ok) return FA_ERR_CUDA;
   // The kernel hands registers between its warpgroups with setmaxnreg; the
   // split only fits if the launch allots kRegsLaunch registers per thread
   // (otherwise setmaxnreg.inc could never be satisfied).
   static int launch_regs = [] {
     cudaFuncAttributes a;
-    return cudaFuncGetAttributes(&a, prefill_kernel<D, GENERAL>) == cudaSuccess ? a.numRegs : -1;
+    return cudaFuncGetAttributes(&a, prefill_kernel<D, GENERAL, FP8>) == cudaSuccess ? a.numRegs : -1;
   }();
   if (launch_regs < (int)kRegsLaunch) return FA_ERR_UNSUPPORTED;
-  prefill_kernel<D, GENERAL><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, GENERAL, FP8><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -316,6 +321,31 @@ fa_status fa_prefill_ex(const void* q, const void* k, const void* v, void* o, fl
                                          s, total_tokens, max_seqlen, var)
              : launch_prefill<128, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
                                           s, total_tokens, max_seqlen, var);
+}
+
+fa_status fa_prefill_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const int32_t* cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                         float scale, float q_descale, float k_descale, float v_descale,
+                         fa_stream_t stream, int total_tokens, int max_seqlen) {
+  if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0 || max_seqlen < 0)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(cu_seqlens, 4) || (lse && !aligned(lse, 4)))
+    return FA_ERR_INVALID_ARG;
+  for (float x : {q_descale, k_descale, v_descale})
+    if (!(x > 0.f) || std::isinf(x)) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hq > 0xFFFF) return FA_ERR_UNSUPPORTED;
+  if ((long long)(max_seqlen + fa::prefill::ROWS_PER_ITEM - 1) / fa::prefill::ROWS_PER_ITEM >
+      fa::prefill::MAX_LEVELS)
+    return FA_ERR_UNSUPPORTED;
+  if (B == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
+  Variant var;
+  var.wr = causal ? 0 : -1;
+  return launch_prefill<128, false, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
+                                          reinterpret_cast<cudaStream_t>(stream), total_tokens,
+                                          max_seqlen, var, q_descale * k_descale, v_descale);
 }
 
 fa_status fa_prefill(const void* q, const void* k, const void* v, void* o, float* lse,

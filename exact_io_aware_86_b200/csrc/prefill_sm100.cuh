@@ -53,6 +53,15 @@
 // In this form a row can see no key at all in its first K/V tile (the band
 // starts inside the tile), so its running max may start at -inf; the exp
 // argument and the rescale factor are guarded for that.
+//
+// FP8 (a third instantiation, FP8 = true; causal or full mask): Q, K and V
+// are e4m3 bytes with per-tensor descale factors.  Both products run as
+// tcgen05 kind::f8f6f4 MMAs (K steps of 32 elements = 32 bytes, so a d=128
+// row is one 128-byte swizzle panel and a tile is 16 KB).  P is rounded to
+// e4m3 (P <= 256 by the lazy rescale, within e4m3's 448) and packed four per
+// tensor-memory column; the row sum that normalises O adds the decoded e4m3
+// values, the LSE sum the unrounded ones.  q_descale * k_descale joins the
+// softmax scale and v_descale the epilogue's 1/l.
 #pragma once
 
 #include "ptx.cuh"
@@ -79,19 +88,85 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int MAX_LEVELS = 1024;  // max_seqlen <= 1024 * 256
 constexpr int MAX_ITEMS_PER_CTA = 256;
 
-template <int D>
+// Instruction descriptor for e4m3 x e4m3 -> fp32 (kind::f8f6f4): the A and
+// B format fields (bits 7-9, 10-12) are 0 for E4M3; the rest as for bf16.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major,
+                                                      bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int D, bool FP8 = false>
 struct Cfg {
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-  static constexpr int PANELS = D / 64;              // 64-element (128 B) swizzle panels
-  static constexpr int PANEL_BYTES = BM * 128;       // 128 rows x 128 B
-  static constexpr int TILE_BYTES = BM * D * 2;      // one Q, K or V tile
-  static constexpr int STAGES = (D == 128) ? 4 : 8;  // K/V ring slots
+  static_assert(!FP8 || D == 128, "the e4m3 path takes head_dim 128");
+  static constexpr int ESIZE = FP8 ? 1 : 2;           // bytes per element
+  static constexpr int PANEL_ELEMS = 128 / ESIZE;     // elements per 128-byte swizzle row
+  static constexpr int PANELS = D / PANEL_ELEMS;      // swizzle panels per tile row
+  static constexpr int PANEL_BYTES = BM * 128;        // 128 rows x 128 B
+  static constexpr int TILE_BYTES = BM * D * ESIZE;   // one Q, K or V tile
+  static constexpr int STAGES = TILE_BYTES <= 16384 ? 8 : 4;  // K/V ring slots
+  static constexpr int KSTEP = 32 / ESIZE;            // K elements per MMA (32 bytes)
+  static constexpr int S_KSTEPS = D / KSTEP;          // MMAs per S tile
+  static constexpr int PV_KSTEPS = BN / KSTEP;        // MMAs per P V tile
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = NQT * TILE_BYTES;
   static constexpr int SMEM_TILES = KV_OFF + STAGES * TILE_BYTES;
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
-  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+  static constexpr uint32_t IDESC_S =
+      FP8 ? idesc_e4m3_f32(BM, BN, false, false) : idesc_bf16_f32(BM, BN, false, false);
+  static constexpr uint32_t IDESC_PV =
+      FP8 ? idesc_e4m3_f32(BM, D, false, true) : idesc_bf16_f32(BM, D, false, true);
 };
+
+// D[tmem] (+)= A * B with e4m3 operands; A from shared memory or tensor memory
+__device__ __forceinline__ void umma_ss_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_e4m3(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+template <bool FP8>
+__device__ __forceinline__ void umma_ss_k(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  if constexpr (FP8) umma_ss_e4m3(d, a, b, id, acc); else umma_ss(d, a, b, id, acc);
+}
+template <bool FP8>
+__device__ __forceinline__ void umma_ts_k(uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  if constexpr (FP8) umma_ts_e4m3(d, a, b, id, acc); else umma_ts(d, a, b, id, acc);
+}
+
+// Two floats -> two e4m3 bytes (nearest, saturating to +-448) in the low 16
+// bits; lo goes to the lower byte (the lower K index).
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// a0 += lower e4m3 value, a1 += upper (exactly: e4m3 -> f16 is exact)
+__device__ __forceinline__ void add_e4m3x2_f32(uint32_t pq, float& a0, float& a1) {
+  asm("{\n\t.reg .b16 q, h0, h1;\n\t.reg .b32 h2;\n\tcvt.u16.u32 q, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h2, q;\n\tmov.b32 {h0, h1}, h2;\n\t"
+      "add.rn.f32.f16 %0, h0, %0;\n\tadd.rn.f32.f16 %1, h1, %1;\n\t}"
+      : "+f"(a0), "+f"(a1) : "r"(pq));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
 
 struct Shared {
   uint64_t q_full, q_empty, mma_done;
@@ -106,9 +181,9 @@ struct Shared {
   int2 items[MAX_ITEMS_PER_CTA];     // (b, level << 16 | h)
 };
 
-template <int D>
+template <int D, bool FP8 = false>
 constexpr int smem_bytes() {
-  return Cfg<D>::SMEM_TILES + (int)sizeof(Shared) + 1024;
+  return Cfg<D, FP8>::SMEM_TILES + (int)sizeof(Shared) + 1024;
 }
 
 struct Params {
@@ -123,6 +198,7 @@ struct Params {
   // wr = 0 under the causal mask.  Every kernel instantiation honours the
   // band's tile range; only GENERAL masks inside tiles by wl / wr.
   int wl, wr;
+  float o_scale;        // multiplies O / l in the epilogue (v_descale; 1 for bf16)
   float cap_in;         // 2 * log2(e) * scale / softcap (GENERAL, softcap > 0)
   float cap_out;        // softcap * log2(e); 0 = no softcap
   const float* alibi;   // ALiBi slopes (GENERAL), or null
@@ -202,11 +278,12 @@ __device__ void decode_item(const Params& p, const Shared& sh, int w, int& b, in
   }
 }
 
-template <int D, bool GENERAL>
+template <int D, bool GENERAL, bool FP8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const Params p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, FP8>;
+  static_assert(!(GENERAL && FP8), "mask variants are not built for e4m3");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -326,7 +403,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const CUtensorMap* m = (next & 1) ? &tmV : &tmK;
 #pragma unroll
             for (int pn = 0; pn < C::PANELS; ++pn)
-              tma_load_2d(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot], kh * D + pn * 64,
+              tma_load_2d(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot], kh * D + pn * C::PANEL_ELEMS,
                           start + (jlo + (next >> 1)) * BN);
             ++kv_it;
           }
@@ -344,7 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int t = 0; t < NQT; ++t)
 #pragma unroll
             for (int pn = 0; pn < C::PANELS; ++pn)
-              tma_prefetch_l2_2d(&tmQ, nh * D + pn * 64, nq0 + t * BM);
+              tma_prefetch_l2_2d(&tmQ, nh * D + pn * C::PANEL_ELEMS, nq0 + t * BM);
         }
         if (!mbar_wait(&sh.q_empty, (q_it & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&sh.q_full, NQT * C::TILE_BYTES);
@@ -353,7 +430,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int pn = 0; pn < C::PANELS; ++pn)
             tma_load_2d(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full,
-                        h * D + pn * 64, start + q0 + t * BM);
+                        h * D + pn * C::PANEL_ELEMS, start + q0 + t * BM);
         ++q_it;
         if (!issue_kv(2 * njobs)) break;
       }
@@ -382,10 +459,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto issue_pv = [&](int t, uint32_t v_idx, bool first) {
         const uint64_t vd = sdesc_advance(v_desc, (v_idx % C::STAGES) * C::TILE_BYTES);
         const uint32_t d_tmem = tmem + 256 + t * 128, a_tmem = tmem + t * 128;
-        umma_ts(d_tmem, a_tmem, vd, C::IDESC_PV, first ? 0u : 1u);
+        // K step kk: 16 (bf16) or 32 (e4m3) keys = 8 tensor-memory columns of
+        // P and KSTEP rows of 128 B of V
+        umma_ts_k<FP8>(d_tmem, a_tmem, vd, C::IDESC_PV, first ? 0u : 1u);
 #pragma unroll
-        for (int kk = 1; kk < BN / 16; ++kk)
-          umma_ts(d_tmem, a_tmem + kk * 8, sdesc_advance(vd, kk * 16 * 128), C::IDESC_PV, 1u);
+        for (int kk = 1; kk < C::PV_KSTEPS; ++kk)
+          umma_ts_k<FP8>(d_tmem, a_tmem + kk * 8, sdesc_advance(vd, kk * C::KSTEP * 128),
+                         C::IDESC_PV, 1u);
       };
       // S_t = Q_t K^T   (both K-major)
       auto issue_s = [&](int t, uint32_t k_idx) {
@@ -393,10 +473,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t kd = sdesc_advance(k_desc, (k_idx % C::STAGES) * C::TILE_BYTES);
         const uint32_t d_tmem = tmem + t * 128;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-          umma_ss(d_tmem, sdesc_advance(qd, off), sdesc_advance(kd, off), C::IDESC_S,
-                  kk > 0 ? 1u : 0u);
+          umma_ss_k<FP8>(d_tmem, sdesc_advance(qd, off), sdesc_advance(kd, off), C::IDESC_S,
+                         kk > 0 ? 1u : 0u);
         }
       };
       for (int it = 0; it < num_items && ok; ++it) {
@@ -602,6 +682,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t neg2 = f2_pack(-m_use, -m_use);
         // GENERAL: s already holds scaled logits, so the FMA multiplies by 1
         const uint64_t mul2 = GENERAL ? f2_pack(1.f, 1.f) : sl2;
+        uint32_t e4_lo = 0;  // e4m3: the even pair of a word, waiting for the odd one
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -618,20 +699,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             float p0, p1;
             f2_unpack(pr, p0, p1);
-            const uint32_t pp = pack_bf16x2(p0, p1);
-            if ((e >> 1) & 1) {
-              le_b = f2_add(le_b, pr);
-              lr_b0 = add_bf16lo_f32(pp, lr_b0);
-              lr_b1 = add_bf16hi_f32(pp, lr_b1);
+            if constexpr (FP8) {
+              // four e4m3 per word: pairs 2w and 2w+1 of the chunk form word w
+              const uint32_t pq = pack_e4m3x2(p0, p1);
+              if ((e >> 1) & 1) {
+                le_b = f2_add(le_b, pr);
+                add_e4m3x2_f32(pq, lr_b0, lr_b1);
+                s[c][e >> 2] = e4_lo | (pq << 16);
+              } else {
+                le_a = f2_add(le_a, pr);
+                add_e4m3x2_f32(pq, lr_a0, lr_a1);
+                e4_lo = pq;
+              }
             } else {
-              le_a = f2_add(le_a, pr);
-              lr_a0 = add_bf16lo_f32(pp, lr_a0);
-              lr_a1 = add_bf16hi_f32(pp, lr_a1);
+              const uint32_t pp = pack_bf16x2(p0, p1);
+              if ((e >> 1) & 1) {
+                le_b = f2_add(le_b, pr);
+                lr_b0 = add_bf16lo_f32(pp, lr_b0);
+                lr_b1 = add_bf16hi_f32(pp, lr_b1);
+              } else {
+                le_a = f2_add(le_a, pr);
+                lr_a0 = add_bf16lo_f32(pp, lr_a0);
+                lr_a1 = add_bf16hi_f32(pp, lr_a1);
+              }
+              s[c][e >> 1] = pp;
             }
-            s[c][e >> 1] = pp;
           }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_st16(s_col + c * 16, s[c]);
+        for (int c = 0; c < 4; ++c) {
+          if constexpr (FP8)
+            tmem_st8(s_col + c * 8, s[c]);  // 32 keys per 8 columns
+          else
+            tmem_st16(s_col + c * 16, s[c]);
+        }
         if (rescale) {
           // O *= alpha; PV_t(j-1) has completed (it precedes S_t(j) in issue order)
           const uint64_t a2 = f2_pack(alpha, alpha);
@@ -665,7 +765,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float l_exact = (la0 + la1) + (lb0 + lb1);
       const float l_round = (lr_a0 + lr_a1) + (lr_b0 + lr_b1);
       const bool valid = qpos < len;
-      const float inv_l = 1.f / l_round;
+      const float inv_l = p.o_scale / l_round;
       const size_t grow = (size_t)(start + qpos);
       uint4* dst = reinterpret_cast<uint4*>(p.o + (grow * p.Hq + h) * D);
 #pragma unroll

@@ -207,6 +207,7 @@ WORKLOADS = {
                       "Hq=32 Hkv=8 d=128",
     "softcap_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 with softcap 50",
     "alibi_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 with ALiBi slopes",
+    "fp8_prefill": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128, Q/K/V in e4m3",
     # inference KV cache step (skill page section 3.5)
     "append_decode": "paged decode with cache append + RoPE (rotary_dim 128), 64 requests, "
                      "Hq=32 Hkv=8 d=128, ctx~U[1024,32767], page 16",
@@ -243,6 +244,26 @@ def varlen_gqa_prefill() -> PrefillInputs:
     return PrefillInputs(name="varlen_gqa_prefill", q=q, k=k, v=v,
                          cu_seqlens=cu_seqlens_of(lengths), lengths=lengths, causal=True,
                          scale=fp32_scale(128), meta={"seed": 1003})
+
+
+def make_prefill_fp8(lengths, Hq: int, Hkv: int, d: int, causal: bool, seed: int,
+                     name: str = "prefill_fp8", spread=(1.0, 1.0, 1.0)) -> PrefillInputs:
+    """e4m3 inputs: fp32 N(0, spread^2) draws rounded to float8_e4m3fn (round to
+    nearest even).  ``meta['descale']`` holds the per-tensor factors (1/spread
+    each) that bring the values back to unit scale."""
+    gen = torch.Generator().manual_seed(seed)
+    T = sum(int(L) for L in lengths)
+    q = (randn_f32((T, Hq, d), gen) * spread[0]).to(torch.float8_e4m3fn)
+    k = (randn_f32((T, Hkv, d), gen) * spread[1]).to(torch.float8_e4m3fn)
+    v = (randn_f32((T, Hkv, d), gen) * spread[2]).to(torch.float8_e4m3fn)
+    return PrefillInputs(name=name, q=q, k=k, v=v, cu_seqlens=cu_seqlens_of(lengths),
+                         lengths=[int(L) for L in lengths], causal=causal, scale=fp32_scale(d),
+                         meta={"seed": seed, "descale": tuple(1.0 / x for x in spread)})
+
+
+def fp8_prefill() -> PrefillInputs:
+    """The causal MHA workload's shape in e4m3 (descale factors 1)."""
+    return make_prefill_fp8([2048] * 4, 16, 16, 128, True, seed=1008, name="fp8_prefill")
 
 
 def window_prefill() -> PrefillInputs:

@@ -113,6 +113,23 @@ fa_status fa_prefill_ex(const void *q, const void *k, const void *v, void *o, fl
                         const float *alibi_slopes, int alibi_batch_stride);
 
 /*
+ * FP8 prefill (the pages list FP8 among the data types of FA3/FA4): q, k, v
+ * are OCP e4m3 bytes (4 exponent bits, bias 7, 3 mantissa bits) in the
+ * layouts of fa_prefill, each with one fp32 descale factor; the operation
+ * is fa_prefill's on the values descale * e4m3.  d must be 128; o is bf16
+ * [T, Hq, d] and lse fp32 [Hq, T] (or NULL) as in fa_prefill.  Both
+ * products run on the tensor cores in e4m3 with fp32 accumulation; the
+ * softmax probabilities are rounded to e4m3 for the second product (relative
+ * error up to 2^-4 each) and O is divided by the sum of those rounded values.
+ * Descale factors must be positive and finite (FA_ERR_INVALID_ARG).
+ * Does not allocate.
+ */
+fa_status fa_prefill_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
+                         const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
+                         float scale, float q_descale, float k_descale, float v_descale,
+                         fa_stream_t stream, int total_tokens, int max_seqlen);
+
+/*
  * Paged decode: one query token per request at the end of its context.
  *
  *   q            bf16 [B, Hq, d]
