@@ -137,14 +137,58 @@ __device__ __forceinline__ void umma_ts_e4m3(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-template <bool FP8>
-__device__ __forceinline__ void umma_ss_k(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-  if constexpr (FP8) umma_ss_e4m3(d, a, b, id, acc); else umma_ss(d, a, b, id, acc);
+// Single-thread instructions issued from a converged warp: elect.sync picks
+// one lane (the lowest, the same every time in a converged warp, so a commit
+// tracks the MMAs that lane issued) and the others skip the instruction.
+// Keeping the issuing warps converged matters: a loop run by lane 0 alone
+// is starved of issue slots when the softmax warps sharing its
+// sub-partition keep the FMA pipe busy (measured: one MMA per ~220 cycles
+// instead of per 64), while a converged loop keeps its pace.
+#define FA_ELECT "{\n\t.reg .pred P, Q;\n\telect.sync _|P, 0xffffffff;\n\t"
+__device__ __forceinline__ void umma_ss_el(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate, bool e4m3) {
+  if (e4m3)
+    asm volatile(FA_ELECT "setp.ne.b32 Q, %4, 0;\n\t"
+                 "@P tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, Q;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+  else
+    asm volatile(FA_ELECT "setp.ne.b32 Q, %4, 0;\n\t"
+                 "@P tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, Q;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
-template <bool FP8>
-__device__ __forceinline__ void umma_ts_k(uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
-  if constexpr (FP8) umma_ts_e4m3(d, a, b, id, acc); else umma_ts(d, a, b, id, acc);
+__device__ __forceinline__ void umma_ts_el(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate, bool e4m3) {
+  if (e4m3)
+    asm volatile(FA_ELECT "setp.ne.b32 Q, %4, 0;\n\t"
+                 "@P tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, Q;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+  else
+    asm volatile(FA_ELECT "setp.ne.b32 Q, %4, 0;\n\t"
+                 "@P tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, Q;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
+__device__ __forceinline__ void commit_el(uint64_t* bar) {
+  asm volatile(FA_ELECT
+               "@P tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void expect_tx_el(uint64_t* bar, uint32_t bytes) {
+  asm volatile(FA_ELECT "@P mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_el(void* dst, const CUtensorMap* m, uint64_t* bar,
+                                               int x, int y) {
+  asm volatile(FA_ELECT
+               "@P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%3, %4}], [%2];\n\t}" ::"r"(smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2_2d_el(const CUtensorMap* m, int x, int y) {
+  asm volatile(FA_ELECT "@P cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];\n\t}"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y) : "memory");
+}
+#undef FA_ELECT
 
 // Two floats -> two e4m3 bytes (nearest, saturating to +-448) in the low 16
 // bits; lo goes to the lower byte (the lower K index).
@@ -378,8 +422,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---- warpgroup 0: producer (warp 0), MMA issuer (warp 1), warps 2-3 idle ----
     setmaxnreg_dec<kRegsControl>();
    if (warp == 0) {
-    // ======================= TMA producer =======================
-    if (lane == 0) {
+    // ================ TMA producer (converged warp, elected issue) ================
+    {
       uint32_t kv_it = 0, q_it = 0;
       for (int it = 0; it < num_items && !*abort; ++it) {
         const int2 item = sh.items[it];
@@ -398,13 +442,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (; next < upto; ++next) {
             const uint32_t slot = kv_it % C::STAGES;
             if (!mbar_wait(&sh.kv_empty[slot], ((kv_it / C::STAGES) & 1) ^ 1, abort)) return false;
-            mbar_arrive_expect_tx(&sh.kv_full[slot], C::TILE_BYTES);
+            expect_tx_el(&sh.kv_full[slot], C::TILE_BYTES);
             uint8_t* dst = kv_smem + slot * C::TILE_BYTES;
             const CUtensorMap* m = (next & 1) ? &tmV : &tmK;
 #pragma unroll
             for (int pn = 0; pn < C::PANELS; ++pn)
-              tma_load_2d(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot], kh * D + pn * C::PANEL_ELEMS,
-                          start + (jlo + (next >> 1)) * BN);
+              tma_load_2d_el(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot],
+                             kh * D + pn * C::PANEL_ELEMS, start + (jlo + (next >> 1)) * BN);
             ++kv_it;
           }
           return true;
@@ -421,16 +465,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int t = 0; t < NQT; ++t)
 #pragma unroll
             for (int pn = 0; pn < C::PANELS; ++pn)
-              tma_prefetch_l2_2d(&tmQ, nh * D + pn * C::PANEL_ELEMS, nq0 + t * BM);
+              tma_prefetch_l2_2d_el(&tmQ, nh * D + pn * C::PANEL_ELEMS, nq0 + t * BM);
         }
         if (!mbar_wait(&sh.q_empty, (q_it & 1) ^ 1, abort)) break;
-        mbar_arrive_expect_tx(&sh.q_full, NQT * C::TILE_BYTES);
+        expect_tx_el(&sh.q_full, NQT * C::TILE_BYTES);
 #pragma unroll
         for (int t = 0; t < NQT; ++t)
 #pragma unroll
           for (int pn = 0; pn < C::PANELS; ++pn)
-            tma_load_2d(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full,
-                        h * D + pn * C::PANEL_ELEMS, start + q0 + t * BM);
+            tma_load_2d_el(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full,
+                           h * D + pn * C::PANEL_ELEMS, start + q0 + t * BM);
         ++q_it;
         if (!issue_kv(2 * njobs)) break;
       }
@@ -443,8 +487,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (q_it > 0) mbar_wait_bounded(&sh.q_full, (q_it - 1) & 1);
     }
    } else if (warp == 1) {
-    // ======================= MMA issuer =======================
-    if (lane == 0) {
+    // ================ MMA issuer (converged warp, elected issue) ================
+    {
       const uint32_t q_addr = smem_u32(q_smem);
       const uint32_t kv_addr = smem_u32(kv_smem);
       uint32_t kv_it = 0, q_it = 0;
@@ -461,11 +505,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem + 256 + t * 128, a_tmem = tmem + t * 128;
         // K step kk: 16 (bf16) or 32 (e4m3) keys = 8 tensor-memory columns of
         // P and KSTEP rows of 128 B of V
-        umma_ts_k<FP8>(d_tmem, a_tmem, vd, C::IDESC_PV, first ? 0u : 1u);
+        umma_ts_el(d_tmem, a_tmem, vd, C::IDESC_PV, first ? 0u : 1u, FP8);
 #pragma unroll
         for (int kk = 1; kk < C::PV_KSTEPS; ++kk)
-          umma_ts_k<FP8>(d_tmem, a_tmem + kk * 8, sdesc_advance(vd, kk * C::KSTEP * 128),
-                         C::IDESC_PV, 1u);
+          umma_ts_el(d_tmem, a_tmem + kk * 8, sdesc_advance(vd, kk * C::KSTEP * 128), C::IDESC_PV,
+                     1u, FP8);
       };
       // S_t = Q_t K^T   (both K-major)
       auto issue_s = [&](int t, uint32_t k_idx) {
@@ -475,8 +519,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-          umma_ss_k<FP8>(d_tmem, sdesc_advance(qd, off), sdesc_advance(kd, off), C::IDESC_S,
-                         kk > 0 ? 1u : 0u);
+          umma_ss_el(d_tmem, sdesc_advance(qd, off), sdesc_advance(kd, off), C::IDESC_S,
+                     kk > 0 ? 1u : 0u, FP8);
         }
       };
       for (int it = 0; it < num_items && ok; ++it) {
@@ -521,11 +565,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             p_phase0 ^= 1;
             tc_fence_after();
             issue_pv(0, v_idx, j == lo0 + 1);
-            if (j == hi0) umma_commit(&sh.o_full[0]);
+            if (j == hi0) commit_el(&sh.o_full[0]);
           }
           if (j >= lo0 && j < hi0) {
             issue_s(0, k_idx);
-            umma_commit(&sh.s_full[0]);
+            commit_el(&sh.s_full[0]);
           }
           // query tile 1
           if (j > lo1 && j <= hi1) {
@@ -533,20 +577,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             p_phase1 ^= 1;
             tc_fence_after();
             issue_pv(1, v_idx, j == lo1 + 1);
-            if (j == hi1) umma_commit(&sh.o_full[1]);
+            if (j == hi1) commit_el(&sh.o_full[1]);
           }
           if (j >= lo1 && j < hi1) {
             issue_s(1, k_idx);
-            umma_commit(&sh.s_full[1]);
+            commit_el(&sh.s_full[1]);
           }
-          if (j > jlo) umma_commit(&sh.kv_empty[v_idx % C::STAGES]);
-          if (j < jhi) umma_commit(&sh.kv_empty[k_idx % C::STAGES]);
-          if (j == jhi - 1 || jhi == jlo) umma_commit(&sh.q_empty);  // last S of the item issued
+          if (j > jlo) commit_el(&sh.kv_empty[v_idx % C::STAGES]);
+          if (j < jhi) commit_el(&sh.kv_empty[k_idx % C::STAGES]);
+          if (j == jhi - 1 || jhi == jlo) commit_el(&sh.q_empty);  // last S of the item issued
         }
         kv_it = base + 2 * (jhi - jlo);
       }
       // every MMA issued must finish before TMEM is released
-      umma_commit(&sh.mma_done);
+      commit_el(&sh.mma_done);
       mbar_wait_bounded(&sh.mma_done, 0);
     }
    }
