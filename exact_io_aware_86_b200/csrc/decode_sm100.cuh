@@ -220,48 +220,57 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
   const int total = (p.split_prefix ? __ldg(p.split_prefix + p.B) : p.B) * p.ngroups;
 
   if (warp == nconsumers) {
-    // ======================= producer =======================
+    // ======================= producer (converged warp) =======================
+    // The whole warp runs the loop: the block-table entries of 32 stages are
+    // fetched at once, one per lane, and broadcast by shuffle, so no stage
+    // waits on a dependent global load; one elected lane issues the copies.
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int g = 0;  // stages issued so far (ring position)
-      bool ok = true;
-      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-        int b, s, y, tb, te, nr;
-        item_of(p, i, b, s, y);
-        item_tokens(p, b, s, tb, te, nr);
-        const int kvh0 = y * p.hpb;
-        const int32_t* bt = p.block_table + (size_t)b * p.max_blocks;
-        const int nst = te > tb ? (te - tb + TOK - 1) / TOK : 0;
-        for (int st = 0; st < nst; ++st, ++g) {
-          const int slot = g % STAGES;
-          if (!mbar_wait(&empty[slot], ((g / STAGES) & 1) ^ 1, abort)) { ok = false; break; }
-          // page_size is a multiple of TOK, so a stage never crosses a page
-          const int t0 = tb + st * TOK;
-          const int page = __ldg(bt + t0 / p.page_size);
-          int z;
-          if (page < 0 || page >= p.num_pages) {
-            report_error(kDevErrBounds);
-            z = -TOK;  // whole box outside the pool: TMA fills zeros
-          } else {
-            z = page * p.page_size + (t0 % p.page_size);
-          }
-          mbar_arrive_expect_tx(&full[slot], 2 * p.half_bytes);
-          uint8_t* kdst = smem + slot * sbytes;
-          uint8_t* vdst = kdst + p.half_bytes;
-          // one box per 64-wide half of head_dim holds all the CTA's kv heads
-          for (int pn = 0; pn < C::PANELS; ++pn) {
-            const int off = pn * p.hpb * BOX_BYTES;
-            tma_load_3d(kdst + off, &tmK, &full[slot], pn * 64, z, kvh0);
-            tma_load_3d(vdst + off, &tmV, &full[slot], pn * 64, z, kvh0);
-          }
+    }
+    __syncwarp();
+    int g = 0;  // stages issued so far (ring position)
+    bool ok = true;
+    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+      int b, s, y, tb, te, nr;
+      item_of(p, i, b, s, y);
+      item_tokens(p, b, s, tb, te, nr);
+      const int kvh0 = y * p.hpb;
+      const int32_t* bt = p.block_table + (size_t)b * p.max_blocks;
+      const int nst = te > tb ? (te - tb + TOK - 1) / TOK : 0;
+      int page_of_lane = 0;
+      for (int st = 0; st < nst; ++st, ++g) {
+        if ((st & 31) == 0) {
+          const int sl = st + lane;  // the stage whose page this lane looks up
+          page_of_lane = sl < nst ? __ldg(bt + (tb + sl * TOK) / p.page_size) : 0;
+        }
+        const int page = __shfl_sync(0xffffffffu, page_of_lane, st & 31);
+        const int slot = g % STAGES;
+        if (!mbar_wait(&empty[slot], ((g / STAGES) & 1) ^ 1, abort)) { ok = false; break; }
+        // page_size is a multiple of TOK, so a stage never crosses a page
+        const int t0 = tb + st * TOK;
+        int z;
+        if (page < 0 || page >= p.num_pages) {
+          if (lane == 0) report_error(kDevErrBounds);
+          z = -TOK;  // whole box outside the pool: TMA fills zeros
+        } else {
+          z = page * p.page_size + (t0 % p.page_size);
+        }
+        expect_tx_el(&full[slot], 2 * p.half_bytes);
+        uint8_t* kdst = smem + slot * sbytes;
+        uint8_t* vdst = kdst + p.half_bytes;
+        // one box per 64-wide half of head_dim holds all the CTA's kv heads
+        for (int pn = 0; pn < C::PANELS; ++pn) {
+          const int off = pn * p.hpb * BOX_BYTES;
+          tma_load_3d_el(kdst + off, &tmK, &full[slot], pn * 64, z, kvh0);
+          tma_load_3d_el(vdst + off, &tmV, &full[slot], pn * 64, z, kvh0);
         }
       }
-      // every load issued must land before the CTA exits
-      for (int s = 0; s < STAGES && s < g; ++s) {
-        const int last = g - 1 - ((g - 1 - s) % STAGES);
-        mbar_wait_bounded(&full[last % STAGES], (last / STAGES) & 1);
-      }
+    }
+    // every load issued must land before the CTA exits
+    for (int s = 0; s < STAGES && s < g; ++s) {
+      const int last = g - 1 - ((g - 1 - s) % STAGES);
+      mbar_wait_bounded(&full[last % STAGES], (last / STAGES) & 1);
     }
   } else {
     // ======================= consumers: one warp per kv head =======================

@@ -137,13 +137,8 @@ __device__ __forceinline__ void umma_ts_e4m3(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Single-thread instructions issued from a converged warp: elect.sync picks
-// one lane (the lowest, the same every time in a converged warp, so a commit
-// tracks the MMAs that lane issued) and the others skip the instruction.
-// Keeping the issuing warps converged matters: a loop run by lane 0 alone
-// is starved of issue slots when the softmax warps sharing its
-// sub-partition keep the FMA pipe busy (measured: one MMA per ~220 cycles
-// instead of per 64), while a converged loop keeps its pace.
+// MMAs issued from a converged warp by one elected lane (see the elected
+// helpers in ptx.cuh for why the issuing warps stay converged).
 #define FA_ELECT "{\n\t.reg .pred P, Q;\n\telect.sync _|P, 0xffffffff;\n\t"
 __device__ __forceinline__ void umma_ss_el(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate, bool e4m3) {
@@ -166,27 +161,6 @@ __device__ __forceinline__ void umma_ts_el(uint32_t d_tmem, uint32_t a_tmem, uin
     asm volatile(FA_ELECT "setp.ne.b32 Q, %4, 0;\n\t"
                  "@P tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, Q;\n\t}" ::"r"(d_tmem),
                  "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
-__device__ __forceinline__ void commit_el(uint64_t* bar) {
-  asm volatile(FA_ELECT
-               "@P tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
-               ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void expect_tx_el(uint64_t* bar, uint32_t bytes) {
-  asm volatile(FA_ELECT "@P mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}"
-               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void tma_load_2d_el(void* dst, const CUtensorMap* m, uint64_t* bar,
-                                               int x, int y) {
-  asm volatile(FA_ELECT
-               "@P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-               " [%0], [%1, {%3, %4}], [%2];\n\t}" ::"r"(smem_u32(dst)),
-               "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_l2_2d_el(const CUtensorMap* m, int x, int y) {
-  asm volatile(FA_ELECT "@P cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];\n\t}"
-               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y) : "memory");
 }
 #undef FA_ELECT
 
