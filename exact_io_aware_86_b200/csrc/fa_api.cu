@@ -107,12 +107,16 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
                          float qk_descale = 1.f, float v_descale = 1.f) {
   using namespace fa::prefill;
   using C = Cfg<D, FP8>;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const cuuint32_t box[2] = {(cuuint32_t)C::PANEL_ELEMS, (cuuint32_t)BM};  // 128 B x 128 rows
   {
     const cuuint64_t dims[2] = {(cuuint64_t)Hq * D, (cuuint64_t)T};
     const cuuint64_t str[1] = {(cuuint64_t)Hq * D * C::ESIZE};
     if (!make_map(&tq, q, 2, dims, str, box, FP8)) return FA_ERR_CUDA;
+    // O is bf16 whatever the input type: 64-column x 128-row store boxes
+    const cuuint64_t ostr[1] = {(cuuint64_t)Hq * D * 2};
+    const cuuint32_t obox[2] = {64, (cuuint32_t)BM};
+    if (!make_map(&to, o, 2, dims, ostr, obox)) return FA_ERR_CUDA;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)Hkv * D, (cuuint64_t)T};
@@ -159,7 +163,7 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
     return cudaFuncGetAttributes(&a, prefill_kernel<D, GENERAL, FP8>) == cudaSuccess ? a.numRegs : -1;
   }();
   if (launch_regs < (int)kRegsLaunch) return FA_ERR_UNSUPPORTED;
-  prefill_kernel<D, GENERAL, FP8><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, GENERAL, FP8><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -86,7 +86,8 @@ static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= NUM_THREADS * kRegsLaun
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int MAX_LEVELS = 1024;  // max_seqlen <= 1024 * 256
-constexpr int MAX_ITEMS_PER_CTA = 256;
+constexpr int MAX_ITEMS_PER_CTA = 192;
+constexpr int SMEM_LIMIT = 232448;  // dynamic shared memory per CTA on sm_100
 
 // Instruction descriptor for e4m3 x e4m3 -> fp32 (kind::f8f6f4): the A and
 // B format fields (bits 7-9, 10-12) are 0 for E4M3; the rest as for bf16.
@@ -111,7 +112,12 @@ struct Cfg {
   static constexpr int PV_KSTEPS = BN / KSTEP;        // MMAs per P V tile
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = NQT * TILE_BYTES;
-  static constexpr int SMEM_TILES = KV_OFF + STAGES * TILE_BYTES;
+  // O leaves through a bf16 staging panel per query tile (64 columns x 128
+  // rows, 128-byte swizzle), one TMA store per panel
+  static constexpr int O_PANEL_BYTES = BM * 128;
+  static constexpr int O_PANELS = D / 64;
+  static constexpr int O_STAGE_OFF = KV_OFF + STAGES * TILE_BYTES;
+  static constexpr int SMEM_TILES = O_STAGE_OFF + NQT * O_PANEL_BYTES;
   static constexpr uint32_t IDESC_S =
       FP8 ? idesc_e4m3_f32(BM, BN, false, false) : idesc_bf16_f32(BM, BN, false, false);
   static constexpr uint32_t IDESC_PV =
@@ -187,22 +193,34 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
 }
 
 struct Shared {
-  uint64_t q_full, q_empty, mma_done;
+  uint64_t q_full[NQT], q_empty[NQT], mma_done;  // Q: one barrier pair per query tile
   uint64_t kv_full[8], kv_empty[8];
   uint64_t s_full[NQT], p_full[NQT], o_full[NQT];
+  // O staging panel of each query tile: written by the tile's 128 threads
+  // (stage_full), read out by the TMA store (stage_free)
+  uint64_t stage_full[NQT], stage_free[NQT];
   uint32_t tmem_base;
   int abort;
   int num_items;                     // items this CTA processes
   int total_items;
+  int2 items[MAX_ITEMS_PER_CTA];     // (b, level << 16 | h)
+};
+
+// Work-list construction scratch; only live before the main loop, so it
+// shares its shared memory with the O staging panels.
+struct PlanScratch {
   int level_count[MAX_LEVELS];       // sequences with more than l 256-row blocks
   int level_offset[MAX_LEVELS + 1];  // first item index of level (descending order)
-  int2 items[MAX_ITEMS_PER_CTA];     // (b, level << 16 | h)
 };
 
 template <int D, bool FP8 = false>
 constexpr int smem_bytes() {
+  static_assert(sizeof(PlanScratch) <= NQT * Cfg<D, FP8>::O_PANEL_BYTES, "plan scratch overflows");
   return Cfg<D, FP8>::SMEM_TILES + (int)sizeof(Shared) + 1024;
 }
+static_assert(smem_bytes<128>() <= SMEM_LIMIT && smem_bytes<64>() <= SMEM_LIMIT &&
+                  smem_bytes<128, true>() <= SMEM_LIMIT,
+              "shared memory layout exceeds the per-CTA limit");
 
 struct Params {
   __nv_bfloat16* o;
@@ -268,7 +286,8 @@ __device__ __forceinline__ int blocks_of(int len) { return (len + ROWS_PER_ITEM 
 
 // Work item w -> (b, level, h).  Items are ordered by descending level
 // (longest causal work first); within a level by sequence, then head.
-__device__ void decode_item(const Params& p, const Shared& sh, int w, int& b, int& level, int& h) {
+__device__ void decode_item(const Params& p, const PlanScratch& sh, int w, int& b, int& level,
+                            int& h) {
   // level_offset[k] is the first item of level num_levels-1-k; find the
   // last k whose offset is <= w (empty levels share their successor's offset)
   int a = 0, z = p.num_levels - 1;
@@ -299,7 +318,8 @@ __device__ void decode_item(const Params& p, const Shared& sh, int w, int& b, in
 template <int D, bool GENERAL, bool FP8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const Params p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const Params p) {
   using C = Cfg<D, FP8>;
   static_assert(!(GENERAL && FP8), "mask variants are not built for e4m3");
   extern __shared__ uint8_t smem_raw[];
@@ -307,7 +327,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                              ~uintptr_t(1023));
   uint8_t* q_smem = smem + C::Q_OFF;
   uint8_t* kv_smem = smem + C::KV_OFF;
+  uint8_t* o_stage = smem + C::O_STAGE_OFF;
   Shared& sh = *reinterpret_cast<Shared*>(smem + C::SMEM_TILES);
+  PlanScratch& ps = *reinterpret_cast<PlanScratch*>(o_stage);
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -315,8 +337,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   // ---------------- prologue: barriers, TMEM, work list ----------------
   if (tid == 0) {
-    mbar_init(&sh.q_full, 1);
-    mbar_init(&sh.q_empty, 1);
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(&sh.q_full[t], 1);
+      mbar_init(&sh.q_empty[t], 1);
+    }
     mbar_init(&sh.mma_done, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&sh.kv_full[s], 1);
@@ -326,6 +350,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&sh.s_full[t], 1);
       mbar_init(&sh.p_full[t], BM);
       mbar_init(&sh.o_full[t], 1);
+      mbar_init(&sh.stage_full[t], BM);
+      mbar_init(&sh.stage_free[t], 1);
     }
     sh.abort = 0;
     fence_mbar_init();
@@ -334,12 +360,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  for (int l = tid; l < p.num_levels; l += NUM_THREADS) sh.level_count[l] = 0;
+  for (int l = tid; l < p.num_levels; l += NUM_THREADS) ps.level_count[l] = 0;
   __syncthreads();
   for (int b = tid; b < p.B; b += NUM_THREADS) {
     int st, len;
@@ -352,16 +379,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       nb = p.num_levels;
     }
     // level l holds sequence b for every l < nb
-    for (int l = 0; l < nb; ++l) atomicAdd(&sh.level_count[l], 1);
+    for (int l = 0; l < nb; ++l) atomicAdd(&ps.level_count[l], 1);
   }
   __syncthreads();
   if (tid == 0) {
     int acc = 0;
     for (int k = 0; k < p.num_levels; ++k) {
-      sh.level_offset[k] = acc;
-      acc += sh.level_count[p.num_levels - 1 - k] * p.Hq;
+      ps.level_offset[k] = acc;
+      acc += ps.level_count[p.num_levels - 1 - k] * p.Hq;
     }
-    sh.level_offset[p.num_levels] = acc;
+    ps.level_offset[p.num_levels] = acc;
     sh.total_items = acc;
     // zig-zag assignment: round r takes item r*G + (r even ? c : G-1-c)
     const int G = gridDim.x, c = blockIdx.x;
@@ -382,7 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int G = gridDim.x, c = blockIdx.x;
     const int w = i * G + ((i & 1) ? (G - 1 - c) : c);
     int b, level, h;
-    decode_item(p, sh, w, b, level, h);
+    decode_item(p, ps, w, b, level, h);
     sh.items[i] = make_int2(b, (level << 16) | h);
   }
   tc_fence_before();
@@ -441,14 +468,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int pn = 0; pn < C::PANELS; ++pn)
               tma_prefetch_l2_2d_el(&tmQ, nh * D + pn * C::PANEL_ELEMS, nq0 + t * BM);
         }
-        if (!mbar_wait(&sh.q_empty, (q_it & 1) ^ 1, abort)) break;
-        expect_tx_el(&sh.q_full, NQT * C::TILE_BYTES);
+        // each query tile's buffer is refilled as soon as the previous item's
+        // last Q K^T of that tile has run (tile 0 usually a step before tile 1)
+        bool stop = false;
 #pragma unroll
-        for (int t = 0; t < NQT; ++t)
+        for (int t = 0; t < NQT; ++t) {
+          if (!mbar_wait(&sh.q_empty[t], (q_it & 1) ^ 1, abort)) { stop = true; break; }
+          expect_tx_el(&sh.q_full[t], C::TILE_BYTES);
 #pragma unroll
           for (int pn = 0; pn < C::PANELS; ++pn)
-            tma_load_2d_el(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full,
+            tma_load_2d_el(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full[t],
                            h * D + pn * C::PANEL_ELEMS, start + q0 + t * BM);
+        }
+        if (stop) break;
         ++q_it;
         if (!issue_kv(2 * njobs)) break;
       }
@@ -458,14 +490,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t last = kv_it - 1 - ((kv_it - 1 - s) % C::STAGES);  // last use of slot
         mbar_wait_bounded(&sh.kv_full[last % C::STAGES], (last / C::STAGES) & 1);
       }
-      if (q_it > 0) mbar_wait_bounded(&sh.q_full, (q_it - 1) & 1);
+      if (q_it > 0)
+        for (int t = 0; t < NQT; ++t) mbar_wait_bounded(&sh.q_full[t], (q_it - 1) & 1);
     }
    } else if (warp == 1) {
     // ================ MMA issuer (converged warp, elected issue) ================
     {
       const uint32_t q_addr = smem_u32(q_smem);
       const uint32_t kv_addr = smem_u32(kv_smem);
-      uint32_t kv_it = 0, q_it = 0;
+      uint32_t kv_it = 0;
       uint32_t p_phase0 = 0, p_phase1 = 0;
       bool ok = true;
       // Descriptors of the first Q tile and the first K/V slot; every other
@@ -497,6 +530,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      kk > 0 ? 1u : 0u, FP8);
         }
       };
+      // Lookahead across items: at an item's last step (only tile 1's last
+      // P V left, since tile 1 ends a step after tile 0 under the causal
+      // mask), tile 0's first Q K^T of the next item is issued before the
+      // wait for tile 1's softmax, so the two softmax groups stay staggered
+      // across item boundaries instead of restarting together.  Only the
+      // plain causal / full kernels take it: with the masked variants'
+      // longer softmax it measured slower.
+      bool la_done = false;  // this item's first tile-0 S was issued by the lookahead
       for (int it = 0; it < num_items && ok; ++it) {
         const int2 item = sh.items[it];
         const int b = item.x, level = item.y >> 16;
@@ -510,8 +551,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tile_kv_range(p, q0, len, lo0, hi0);
         if (q0 + BM < len) tile_kv_range(p, q0 + BM, len, lo1, hi1);
         const int jlo = lo0, jhi = max(hi0, hi1);
-        if (!mbar_wait(&sh.q_full, q_it & 1, abort)) { ok = false; break; }
-        ++q_it;
+        // per tile: Q waited for, Q released (each exactly once per item)
+        bool qw0 = la_done, qw1 = false;
+        bool qr0 = la_done && hi0 - lo0 == 1, qr1 = false;
+        const bool skip_s0 = la_done;
+        la_done = false;
         const uint32_t base = kv_it;
         // step j issues P V of tile j-1 and Q K^T of tile j, per query tile
         for (int j = jlo; j <= jhi; ++j) {
@@ -519,9 +563,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // both slots are normally full already: test them together so the
           // two barrier latencies overlap, and block only on a miss
           const bool k_ready = j >= jhi || mbar_try_wait(smem_u32(&sh.kv_full[k_idx % C::STAGES]),
-                                                         (k_idx / C::STAGES) & 1);
+                                                     (k_idx / C::STAGES) & 1);
           const bool v_ready = j <= jlo || mbar_try_wait(smem_u32(&sh.kv_full[v_idx % C::STAGES]),
-                                                         (v_idx / C::STAGES) & 1);
+                                                     (v_idx / C::STAGES) & 1);
           if (!k_ready &&
               !mbar_wait(&sh.kv_full[k_idx % C::STAGES], (k_idx / C::STAGES) & 1, abort)) {
             ok = false;
@@ -541,9 +585,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             issue_pv(0, v_idx, j == lo0 + 1);
             if (j == hi0) commit_el(&sh.o_full[0]);
           }
-          if (j >= lo0 && j < hi0) {
-            issue_s(0, k_idx);
+          // tile 0's Q K^T of this step or, at the item's last step, the
+          // next item's first one (lookahead); never both in one step
+          int s0_idx = -1;       // K slot of tile 0's Q K^T, if any
+          bool s0_last = false;  // it is the last one of its item: release Q0
+          if (j >= lo0 && j < hi0 && !(skip_s0 && j == lo0)) {
+            if (!qw0) {
+              if (!mbar_wait(&sh.q_full[0], it & 1, abort)) { ok = false; break; }
+              qw0 = true;
+            }
+            s0_idx = (int)k_idx;
+            s0_last = j == hi0 - 1;
+            qr0 = qr0 || s0_last;
+          } else if (!GENERAL && j == jhi && hi0 < jhi && qr0 && it + 1 < num_items) {
+            const int2 nx = sh.items[it + 1];
+            int ns, nl;
+            seq_range(p, nx.x, ns, nl);
+            (void)ns;
+            int nlo, nhi;
+            tile_kv_range(p, (nx.y >> 16) * ROWS_PER_ITEM, nl, nlo, nhi);
+            if (nhi > nlo) {
+              const uint32_t nk = base + 2 * (jhi - jlo);  // the next item's first K
+              if (!mbar_wait(&sh.q_full[0], (it + 1) & 1, abort) ||
+                  !mbar_wait(&sh.kv_full[nk % C::STAGES], (nk / C::STAGES) & 1, abort)) {
+                ok = false;
+                break;
+              }
+              s0_idx = (int)nk;
+              s0_last = nhi - nlo == 1;
+              la_done = true;
+            }
+          }
+          if (s0_idx >= 0) {
+            tc_fence_after();
+            issue_s(0, (uint32_t)s0_idx);
             commit_el(&sh.s_full[0]);
+            if (s0_last) commit_el(&sh.q_empty[0]);
           }
           // query tile 1
           if (j > lo1 && j <= hi1) {
@@ -554,13 +631,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (j == hi1) commit_el(&sh.o_full[1]);
           }
           if (j >= lo1 && j < hi1) {
+            if (!qw1) {
+              if (!mbar_wait(&sh.q_full[1], it & 1, abort)) { ok = false; break; }
+              qw1 = true;
+              tc_fence_after();
+            }
             issue_s(1, k_idx);
             commit_el(&sh.s_full[1]);
+            if (j == hi1 - 1) { commit_el(&sh.q_empty[1]); qr1 = true; }
           }
           if (j > jlo) commit_el(&sh.kv_empty[v_idx % C::STAGES]);
           if (j < jhi) commit_el(&sh.kv_empty[k_idx % C::STAGES]);
-          if (j == jhi - 1 || jhi == jlo) commit_el(&sh.q_empty);  // last S of the item issued
         }
+        if (!ok) break;
+        // a tile with no Q K^T in this item (past the sequence end) still
+        // takes its Q phase and releases its buffer, keeping the phases paired
+        if (!qw0 && !mbar_wait(&sh.q_full[0], it & 1, abort)) { ok = false; break; }
+        if (!qr0) commit_el(&sh.q_empty[0]);
+        if (!qw1 && !mbar_wait(&sh.q_full[1], it & 1, abort)) { ok = false; break; }
+        if (!qr1) commit_el(&sh.q_empty[1]);
         kv_it = base + 2 * (jhi - jlo);
       }
       // every MMA issued must finish before TMEM is released
@@ -578,6 +667,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t s_col = lane_base + t * 128;
     const uint32_t o_col = lane_base + 256 + t * 128;
     uint32_t s_phase = 0, o_phase = 0;
+    uint32_t n_stage = 0;  // O panels staged by this group so far
     const float sl = p.scale_log2;
     const uint64_t sl2 = f2_pack(sl, sl);
     bool ok = true;
@@ -785,26 +875,80 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool valid = qpos < len;
       const float inv_l = p.o_scale / l_round;
       const size_t grow = (size_t)(start + qpos);
-      uint4* dst = reinterpret_cast<uint4*>(p.o + (grow * p.Hq + h) * D);
+      if (rs + BM <= len) {
+        // full tile: each 64-column panel is normalised into the staging
+        // panel (row = this thread's row, 16-byte chunks swizzled by row & 7)
+        // and written by one TMA store, so no thread waits on global stores
+        uint8_t* stage = o_stage + t * C::O_PANEL_BYTES;
+        uint8_t* srow = stage + row * 128;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(o_col + c * 32, o);
-        tmem_ld_wait(o);
-        uint32_t w[16];
+        for (int pn = 0; pn < C::O_PANELS; ++pn) {
+          uint32_t o[2][32];
+          tmem_ld32(o_col + pn * 64, o[0]);
+          tmem_ld32(o_col + pn * 64 + 32, o[1]);
+          tmem_ld_wait(o[0]);
+          tmem_ld_wait(o[1]);
+          // the previous store from this panel must have read it out
+          if (n_stage > 0 && !mbar_wait(&sh.stage_free[t], (n_stage - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (valid) {
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* src = o[c >> 2] + (c & 3) * 8;
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(src[0]) * inv_l, __uint_as_float(src[1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(src[2]) * inv_l, __uint_as_float(src[3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(src[4]) * inv_l, __uint_as_float(src[5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(src[6]) * inv_l, __uint_as_float(src[7]) * inv_l);
+            *reinterpret_cast<uint4*>(srow + ((c ^ (row & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&sh.stage_full[t]);
+          bool stored = true;
+          if (row == 0) {
+            stored = mbar_wait(&sh.stage_full[t], n_stage & 1, abort);
+            if (stored) {
+              tma_store_2d(&tmO, stage, h * D + pn * 64, start + rs);
+              bulk_commit_group();
+              bulk_wait_read_all();
+              mbar_arrive(&sh.stage_free[t]);
+            }
+          }
+          ++n_stage;
+          if (!__all_sync(0xffffffffu, stored)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+      } else {
+        // the tile runs past the sequence end: rows are stored one by one
+        // (every lane takes part in the warp-wide TMEM loads)
+        uint4* dst = reinterpret_cast<uint4*>(p.o + (grow * p.Hq + h) * D);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[c * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_col + c * 32, o);
+          tmem_ld_wait(o);
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                               __uint_as_float(o[2 * e + 1]) * inv_l);
+          if (valid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[c * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          }
         }
       }
       if (valid && p.lse)
         p.lse[(size_t)h * p.T + grow] = (m_ref + __log2f(l_exact)) * 0.69314718055994531f;
       tc_fence_before();
     }
+    // the staged O stores must be complete before the CTA exits
+    if (row == 0) bulk_wait_all();
   }
 
   // ---------------- teardown ----------------
