@@ -73,13 +73,15 @@ constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 128;           // keys per K/V tile
 constexpr int NQT = 2;            // query tiles per work item
 constexpr int ROWS_PER_ITEM = NQT * BM;
+constexpr int P_CHUNKS = 2;       // P is handed to the P V MMAs in chunks of BN / P_CHUNKS keys
+static_assert(P_CHUNKS == 1 || P_CHUNKS == 2 || P_CHUNKS == 4, "P chunks are whole 32-key quarters");
 constexpr int NUM_WARPS = 12;  // 3 warpgroups: control (producer, MMA, 2 idle), softmax x2
 constexpr int NUM_THREADS = NUM_WARPS * 32;
 // Register split between the warpgroups (setmaxnreg).  The launch allots
 // kRegsLaunch per thread; the control group gives most of its share to the
 // softmax groups: 128*kRegsControl + 256*kRegsSoftmax <= 384*kRegsLaunch.
 constexpr uint32_t kRegsLaunch = 168;
-constexpr uint32_t kRegsControl = 96;
+constexpr uint32_t kRegsControl = 104;
 constexpr uint32_t kRegsSoftmax = 200;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= NUM_THREADS * kRegsLaunch,
               "register split exceeds the launch allocation");
@@ -195,7 +197,8 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
 struct Shared {
   uint64_t q_full[NQT], q_empty[NQT], mma_done;  // Q: one barrier pair per query tile
   uint64_t kv_full[8], kv_empty[8];
-  uint64_t s_full[NQT], p_full[NQT], o_full[NQT];
+  uint64_t s_full[NQT], o_full[NQT];
+  uint64_t p_full[NQT][P_CHUNKS];  // one chunk of P written to TMEM
   // O staging panel of each query tile: written by the tile's 128 threads
   // (stage_full), read out by the TMA store (stage_free)
   uint64_t stage_full[NQT], stage_free[NQT];
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int t = 0; t < NQT; ++t) {
       mbar_init(&sh.s_full[t], 1);
-      mbar_init(&sh.p_full[t], BM);
+      for (int c = 0; c < P_CHUNKS; ++c) mbar_init(&sh.p_full[t][c], BM);
       mbar_init(&sh.o_full[t], 1);
       mbar_init(&sh.stage_full[t], BM);
       mbar_init(&sh.stage_free[t], 1);
@@ -506,17 +509,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t q_desc = sdesc_sw128(q_addr, 16, 1024);           // K-major
       const uint64_t k_desc = sdesc_sw128(kv_addr, 16, 1024);          // K-major
       const uint64_t v_desc = sdesc_sw128(kv_addr, C::PANEL_BYTES, 1024);  // MN-major
-      // O_t += P_t V   (A = P from TMEM, B = V, MN-major)
-      auto issue_pv = [&](int t, uint32_t v_idx, bool first) {
+      // O_t += P_t V over the keys of P chunk c (A = P from TMEM, B = V,
+      // MN-major); the first chunk of a tile's first step overwrites O
+      constexpr int PV_PER_CHUNK = C::PV_KSTEPS / P_CHUNKS;
+      auto issue_pv = [&](int t, uint32_t v_idx, int c, bool first) {
         const uint64_t vd = sdesc_advance(v_desc, (v_idx % C::STAGES) * C::TILE_BYTES);
         const uint32_t d_tmem = tmem + 256 + t * 128, a_tmem = tmem + t * 128;
         // K step kk: 16 (bf16) or 32 (e4m3) keys = 8 tensor-memory columns of
         // P and KSTEP rows of 128 B of V
-        umma_ts_el(d_tmem, a_tmem, vd, C::IDESC_PV, first ? 0u : 1u, FP8);
 #pragma unroll
-        for (int kk = 1; kk < C::PV_KSTEPS; ++kk)
+        for (int q = 0; q < PV_PER_CHUNK; ++q) {
+          const int kk = c * PV_PER_CHUNK + q;
           umma_ts_el(d_tmem, a_tmem + kk * 8, sdesc_advance(vd, kk * C::KSTEP * 128), C::IDESC_PV,
-                     1u, FP8);
+                     (first && kk == 0) ? 0u : 1u, FP8);
+        }
       };
       // S_t = Q_t K^T   (both K-major)
       auto issue_s = [&](int t, uint32_t k_idx) {
@@ -579,10 +585,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           // query tile 0
           if (j > lo0 && j <= hi0) {
-            if (!mbar_wait(&sh.p_full[0], p_phase0, abort)) { ok = false; break; }
+            // each chunk's MMAs go out as soon as the softmax has stored it
+            bool pv_ok = true;
+#pragma unroll
+            for (int c = 0; c < P_CHUNKS; ++c) {
+              if (!mbar_wait(&sh.p_full[0][c], p_phase0, abort)) { pv_ok = false; break; }
+              tc_fence_after();
+              issue_pv(0, v_idx, c, j == lo0 + 1);
+            }
+            if (!pv_ok) { ok = false; break; }
             p_phase0 ^= 1;
-            tc_fence_after();
-            issue_pv(0, v_idx, j == lo0 + 1);
             if (j == hi0) commit_el(&sh.o_full[0]);
           }
           // tile 0's Q K^T of this step or, at the item's last step, the
@@ -624,10 +636,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           // query tile 1
           if (j > lo1 && j <= hi1) {
-            if (!mbar_wait(&sh.p_full[1], p_phase1, abort)) { ok = false; break; }
+            // each chunk's MMAs go out as soon as the softmax has stored it
+            bool pv_ok = true;
+#pragma unroll
+            for (int c = 0; c < P_CHUNKS; ++c) {
+              if (!mbar_wait(&sh.p_full[1][c], p_phase1, abort)) { pv_ok = false; break; }
+              tc_fence_after();
+              issue_pv(1, v_idx, c, j == lo1 + 1);
+            }
+            if (!pv_ok) { ok = false; break; }
             p_phase1 ^= 1;
-            tc_fence_after();
-            issue_pv(1, v_idx, j == lo1 + 1);
             if (j == hi1) commit_el(&sh.o_full[1]);
           }
           if (j >= lo1 && j < hi1) {
@@ -784,6 +802,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           m_ref = m_new;
           rescale = true;
         }
+        if (rescale) {
+          // O *= alpha before any chunk of P is released: every P V of step j-1
+          // has completed (they precede S_t(j) in issue order).  16 columns at
+          // a time, since all of S is still held in registers here.
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(o_col + c * 16, o);
+            tmem_ld_wait16(o);
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              float o0, o1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
+              o[e] = __float_as_uint(o0);
+              o[e + 1] = __float_as_uint(o1);
+            }
+            tmem_st16(o_col + c * 16, o);
+          }
+        }
         // P = 2^(s*scale*log2e - m): three of every four pairs on MUFU, one on
         // the FMA pipe; packed bf16 pairs overwrite s[c][0..15] in order
         const float m_use = (GENERAL && m_ref == -INFINITY) ? 0.f : m_ref;
@@ -791,8 +829,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // GENERAL: s already holds scaled logits, so the FMA multiplies by 1
         const uint64_t mul2 = GENERAL ? f2_pack(1.f, 1.f) : sl2;
         uint32_t e4_lo = 0;  // e4m3: the even pair of a word, waiting for the odd one
+        // four 32-key quarters; a chunk is 4 / P_CHUNKS consecutive quarters
+        constexpr int QPC = 4 / P_CHUNKS;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const uint64_t x =
@@ -833,34 +873,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               s[c][e >> 1] = pp;
             }
           }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
+          // the chunk that ended with quarter c-1 has had this quarter's math
+          // to land: release it, then store quarter c
+          if (c > 0 && c % QPC == 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sh.p_full[t][c / QPC - 1]);
+          }
           if constexpr (FP8)
             tmem_st8(s_col + c * 8, s[c]);  // 32 keys per 8 columns
           else
             tmem_st16(s_col + c * 16, s[c]);
         }
-        if (rescale) {
-          // O *= alpha; PV_t(j-1) has completed (it precedes S_t(j) in issue order)
-          const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(o_col + c * 32, o);
-            tmem_ld_wait(o);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float o0, o1;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), o0, o1);
-              o[e] = __float_as_uint(o0);
-              o[e + 1] = __float_as_uint(o1);
-            }
-            tmem_st32(o_col + c * 32, o);
-          }
-        }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&sh.p_full[t]);
+        mbar_arrive(&sh.p_full[t][P_CHUNKS - 1]);
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16, LSE ----
