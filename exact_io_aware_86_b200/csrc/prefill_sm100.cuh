@@ -11,11 +11,15 @@
 //   running row max m and sum l, write P = exp(S*scale - m) back into tensor
 //   memory as bf16, and the tensor cores accumulate O += P V_j in tensor
 //   memory.  At the end O / l is stored as bf16 and LSE = ln2*(m + log2 l).
+//   Full tiles of O leave through a swizzled shared-memory staging panel and
+//   TMA stores; a tile that runs past its sequence's end is stored row by row.
 //
 // CTA layout (384 threads = 3 warpgroups, one CTA per SM, persistent):
-//   warp 0      TMA producer: Q tiles once per work item, then K_j, V_j
-//               alternately through a ring of 128 x D smem slots
-//   warp 1      MMA issuer (one thread) and TMEM owner (512 columns)
+//   warp 0      TMA producer: Q tiles once per work item (one barrier pair
+//               per query tile), then K_j, V_j alternately through a ring
+//               of 128 x D smem slots
+//   warp 1      MMA issuer (converged warp, elected lane) and TMEM owner
+//               (512 columns)
 //   warps 2-3   idle (they complete the first warpgroup)
 //   warps 4-7   softmax for query tile 0 (rows q0 .. q0+127)
 //   warps 8-11  softmax for query tile 1 (rows q0+128 .. q0+255)
@@ -26,12 +30,19 @@
 // Tensor memory columns: S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [384,384+D).  P_t (bf16, 2 per column) overwrites the first 64 columns
 // of S_t once S_t has been read; the MMA that writes the next S_t is issued
-// after the P_t V MMA, and tcgen05 MMAs from one thread execute in order.
+// after the P_t V MMAs, and tcgen05 MMAs from one thread execute in order.
+// P is released in two 64-key halves, each on its own barrier, so the first
+// half's P V MMAs run while the softmax still computes the second half.  At
+// an item's last step the MMA warp issues the next item's first S_0 before
+// it waits for tile 1's last P (plain causal / full kernels), so the two
+// softmax groups stay staggered across work items.
 //
 // Lazy rescaling: a row's reference max m only moves when the tile max
 // exceeds it by more than 8 (log2 units), so P <= 256 and O is rescaled in
-// tensor memory only on those (rare) tiles.  The final O / l and the LSE use
-// the same reference max, so the result is exact up to rounding.
+// tensor memory only on those (rare) tiles, before any of the tile's P is
+// released (every P V of the previous step has completed once S is
+// committed).  The final O / l and the LSE use the same reference max, so
+// the result is exact up to rounding.
 //
 // Softmax arithmetic per score: one three-input max per two scores, one
 // packed FMA per two scores for s*scale*log2e - m, 2^x on the MUFU unit for

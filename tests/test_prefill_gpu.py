@@ -81,6 +81,15 @@ def test_varlen(lengths, Hq, Hkv, causal, d):
     assert_prefill_matches(inp)
 
 
+def test_more_items_than_one_cta_holds():
+    """2048 one- and two-token sequences plus two long ones, 16 query heads:
+    about 33k work items, more than 148 CTAs can list, so the launch widens
+    the grid past one CTA per SM.  Every row is checked."""
+    lengths = [1, 2] * 1024 + [1000, 513]
+    inp = inputs.make_prefill(lengths, 16, 4, 128, True, seed=4005)
+    assert_prefill_matches(inp)
+
+
 def test_varlen_equals_separate_calls():
     lengths = [300, 129, 700]
     inp = inputs.make_prefill(lengths, 8, 2, 128, True, seed=4001)
