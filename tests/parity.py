@@ -39,12 +39,14 @@ def check_bf16(got, ref, what="O"):
 
 
 def check_bf16_peaked(got, ref, what="O"):
-    """Bounds for deliberately peaked rows (a window of one or two keys,
-    logits of tens of units): there O is close to a single value row, so |O|
-    reaches 2-5 and bf16 cannot hold it to 1e-2 -- storing O costs up to
-    2^-9 |O|, and the bf16 weights P a further 2^-9 (max|v| + |O|).  The max
-    bound is therefore 1e-2 + 2^-8 |ref| elementwise (one bf16 ulp of the
-    exact value on top of the absolute bound); the mean bound is unchanged."""
+    """Bounds for peaked rows (a window of one or two keys, logits of tens of
+    units, sequences of one or two tokens): there O is close to a single
+    value row, so |O| reaches 2-5 and bf16 cannot hold it to 1e-2.  bf16 has 8
+    significant bits, so rounding O to it errs by up to 2^-8 |O| (0.0156 on
+    [4, 8)); rounding the weights P to bf16 moves O by a further
+    sum_j w_j d_j (v_j - O) / sum w, |d_j| <= 2^-8, which the absolute 1e-2
+    covers.  The max bound is therefore 1e-2 + 2^-8 |ref| elementwise; the
+    mean bound is unchanged."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, f"{what}: shape {got.shape} vs {ref.shape}"
