@@ -72,9 +72,16 @@ typedef enum {
  *               zero: it sees all L_b keys of its own sequence
  *   scale       multiplier of Q K^T (<= 0: 1/sqrt(d))
  *   total_tokens  T (host copy of cu_seqlens[B]; sizes q/k/v/o)
- *   max_seqlen    an upper bound on every L_b (host; sizes the grid)
- * Query head h reads kv head h / (Hq / Hkv).  A sequence with L_b = 0 is
- * skipped.  Does not allocate.
+ *   max_seqlen    an upper bound on every L_b (host): sizes the device work
+ *                 list of 256-row blocks.  At most 262144
+ *                 (FA_ERR_UNSUPPORTED above).  For a sequence longer than
+ *                 ceil(max_seqlen / 256) * 256 rows, the rows past that are
+ *                 not computed (their O and LSE are left as they were) and
+ *                 FA_ERR_DEVICE_BOUNDS is set.
+ * Query head h reads kv head h / (Hq / Hkv); Hq <= 65535.  A sequence with
+ * L_b = 0 is skipped.  The grid is one CTA per SM, widened when a CTA would
+ * have to list more than 192 work items (sequence, 256-row block, head).
+ * Does not allocate.
  */
 fa_status fa_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
                      const int32_t *cu_seqlens, int B, int Hq, int Hkv, int d, int causal,
