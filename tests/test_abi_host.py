@@ -70,6 +70,7 @@ def test_prefill_argument_checks(lib):
     assert _prefill(lib, d=96) == api.FA_ERR_UNSUPPORTED
     assert _prefill(lib, d=256) == api.FA_ERR_UNSUPPORTED
     assert _prefill(lib, maxlen=1024 * 256 + 1) == api.FA_ERR_UNSUPPORTED
+    assert _prefill(lib, Hq=65536, Hkv=1) == api.FA_ERR_UNSUPPORTED   # head index is 16-bit
     # empty problems are a no-op (no launch)
     assert _prefill(lib, B=0) == api.FA_OK
     assert _prefill(lib, T=0) == api.FA_OK
@@ -94,6 +95,30 @@ def test_prefill_ex_argument_checks(lib):
     assert _prefill_ex(lib, d=96, wl=4) == api.FA_ERR_UNSUPPORTED
     # empty problems are a no-op whatever the variant
     assert _prefill_ex(lib, B=0, wl=3, wr=2, cap=30.0, alibi=FAKE, stride=4) == api.FA_OK
+
+
+def _prefill_fp8(lib, qd=1.0, kd=1.0, vd=1.0, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, cu=FAKE, B=1, Hq=4, Hkv=2, d=128,
+             causal=1, scale=0.0, stream=None, T=16, maxlen=16)
+    a.update(kw)
+    return lib.fa_prefill_fp8(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu"], a["B"],
+                              a["Hq"], a["Hkv"], a["d"], a["causal"], a["scale"], qd, kd, vd,
+                              a["stream"], a["T"], a["maxlen"])
+
+
+def test_prefill_fp8_argument_checks(lib):
+    assert _prefill_fp8(lib, v=None) == api.FA_ERR_INVALID_ARG
+    assert _prefill_fp8(lib, Hq=6, Hkv=4) == api.FA_ERR_INVALID_ARG
+    assert _prefill_fp8(lib, o=ctypes.c_void_p(0x1004)) == api.FA_ERR_INVALID_ARG  # misaligned
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        assert _prefill_fp8(lib, qd=bad) == api.FA_ERR_INVALID_ARG
+        assert _prefill_fp8(lib, kd=bad) == api.FA_ERR_INVALID_ARG
+        assert _prefill_fp8(lib, vd=bad) == api.FA_ERR_INVALID_ARG
+    assert _prefill_fp8(lib, d=64) == api.FA_ERR_UNSUPPORTED           # e4m3 path is d = 128
+    assert _prefill_fp8(lib, Hq=65536, Hkv=1) == api.FA_ERR_UNSUPPORTED
+    assert _prefill_fp8(lib, maxlen=1024 * 256 + 1) == api.FA_ERR_UNSUPPORTED
+    assert _prefill_fp8(lib, B=0) == api.FA_OK
+    assert _prefill_fp8(lib, T=0) == api.FA_OK
 
 
 def _decode(lib, **kw):
