@@ -34,7 +34,7 @@ def bf16_rounding_floor(ref):
 
 
 def check_bf16(got, ref, what="O"):
-    """Spec bounds for bf16 outputs (see the module docstring)."""
+    """The bf16 output bounds: max-abs 1e-2, and mean-abs 1e-3 above the rounding floor."""
     return check_close(got, ref, BF16_MAX_ABS, BF16_MEAN_ABS + bf16_rounding_floor(ref), what)
 
 
