@@ -53,3 +53,42 @@ def test_accounting_matches_the_pages_conventions():
     d = inputs.make_decode([17, 32], 4, 2, 16, 16, seed=1)
     # 49 tokens x Hkv 2 x d 16 x 2 B x (K, V); q and o; ceil(17/16) + ceil(32/16) = 4 pages; 2 lengths
     assert bench.decode_bytes(d) == (49 * 2 * 16 * 2 * 2) + 2 * 2 * 4 * 16 * 2 + 4 * 4 + 4 * 2
+
+
+def _pairs_by_mask(L, causal, left, right):
+    """Brute-force count of the (query, key) pairs a mask leaves visible."""
+    n = 0
+    for i in range(L):
+        for j in range(L):
+            if causal and j > i:
+                continue
+            if left >= 0 and j < i - left:
+                continue
+            if right >= 0 and j > i + right:
+                continue
+            n += 1
+    return n
+
+
+@pytest.mark.parametrize("L", [1, 2, 7, 33, 130])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("window", [(-1, -1), (0, 0), (3, -1), (-1, 5), (4, 2), (40, 0), (200, 7)])
+def test_visible_pairs_equal_the_mask(L, causal, window):
+    """The work a prefill workload is credited with counts exactly the pairs
+    the mask (causal and/or window) leaves visible."""
+    import bench
+    assert bench.visible_pairs(L, causal, window) == _pairs_by_mask(L, causal, *window)
+
+
+def test_append_decode_bytes():
+    """An appended token joins the context; the call also moves k_new, v_new
+    (read), the new k, v (written) and one cos and one sin row per request."""
+    import bench
+    from exact_io_aware_86_b200 import inputs
+    a = inputs.make_append_decode([15, 40], 4, 2, 16, 16, seed=2, rotary_dim=8, max_pos=64)
+    ctx = [16, 41]
+    kv = sum(ctx) * 2 * 16 * 2 * 2
+    qo = 2 * 2 * 4 * 16 * 2
+    pages = 1 + 3
+    extra = 2 * (2 * 2 * 2 * 16 * 2) + 2 * 2 * 4 * 4
+    assert bench.decode_bytes(a) == kv + qo + 4 * pages + 4 * 2 + extra
