@@ -15,6 +15,11 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa.so")
 
+# Largest batch whose decode plan (the prefix of per-request range counts)
+# each CTA of the split kernel builds itself; larger batches get it from a
+# separate one-CTA plan kernel (FA_DECODE_PLAN_MAX_B in include/fa.h).
+DECODE_PLAN_MAX_B = 2048
+
 FA_OK = 0
 FA_ERR_INVALID_ARG = 1
 FA_ERR_UNSUPPORTED = 2
@@ -68,6 +73,10 @@ def load_library(path: str = LIB_PATH):
     lib.fa_get_error_string.argtypes = [i32]
     lib.fa_get_error_string.restype = ctypes.c_char_p
     lib.fa_version.argtypes = []
+    lib.fa_selftest_math.argtypes = [i32, vp, vp, i32, f32, f32, vp]
+    lib.fa_selftest_math.restype = ctypes.c_int
+    lib.fa_selftest_inject_stall.argtypes = [i32, ctypes.c_ulonglong]
+    lib.fa_selftest_inject_stall.restype = ctypes.c_int
     for f in (lib.fa_prefill, lib.fa_prefill_ex, lib.fa_decode_paged, lib.fa_decode_auto_splits, lib.fa_prefill_f32,
               lib.fa_decode_paged_f32, lib.fa_get_device_error, lib.fa_version):
         f.restype = ctypes.c_int
@@ -96,17 +105,26 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream))
 
 
-def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int, shape=None) -> None:
+    """Type, dtype, rank, optional exact shape and contiguity of an argument.
+    The device is checked separately (``_on_cuda``), after every shape, so a
+    wrong shape is reported the same way on any device."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be on a CUDA device")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _on_cuda(**tensors) -> None:
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{name} must be on a CUDA device")
 
 
 # --------------------------------------------------------------------------
@@ -137,6 +155,7 @@ def fa_prefill(q, k, v, o, lse, cu_seqlens, causal: bool, scale: float = 0.0,
         raise ValueError("q/k/v/o shapes disagree")
     if lse is not None and lse.shape != (Hq, T):
         raise ValueError("lse must be [Hq, T]")
+    _on_cuda(q=q, k=k, v=v, o=o, lse=lse, cu_seqlens=cu_seqlens, alibi_slopes=alibi_slopes)
     B = cu_seqlens.numel() - 1
     ms = T if max_seqlen is None else int(max_seqlen)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), B, Hq, Hkv, d,
@@ -195,6 +214,7 @@ def fa_prefill_fp8(q, k, v, o, lse, cu_seqlens, causal: bool, scale: float = 0.0
         raise ValueError("q/k/v/o shapes disagree")
     if lse is not None and lse.shape != (Hq, T):
         raise ValueError("lse must be [Hq, T]")
+    _on_cuda(q=q, k=k, v=v, o=o, lse=lse, cu_seqlens=cu_seqlens)
     B = cu_seqlens.numel() - 1
     ms = T if max_seqlen is None else int(max_seqlen)
     _check(load_library().fa_prefill_fp8(
@@ -236,7 +256,11 @@ def decode_auto_splits(B: int, Hq: int, Hkv: int, max_blocks_per_seq: int, page_
                                                     num_sms))
 
 
-def _decode_shapes(q, k_pages, v_pages, block_table, seq_lens, dt):
+def _decode_shapes(q, k_pages, v_pages, block_table, seq_lens, dt, o=None, lse=None,
+                   o_dtype=None):
+    """Checks the decode arguments (o [B, Hq, d] and lse [B, Hq] when given:
+    the kernels write exactly that many elements) and returns the shape
+    scalars (B, Hq, Hkv, d, num_pages, page_size, max_blocks)."""
     _need(q, "q", dt, 3)
     _need(k_pages, "k_pages", dt, 4)
     _need(v_pages, "v_pages", dt, 4)
@@ -248,6 +272,12 @@ def _decode_shapes(q, k_pages, v_pages, block_table, seq_lens, dt):
         raise ValueError("q/k_pages/v_pages shapes disagree")
     if block_table.shape[0] != B or seq_lens.shape[0] != B:
         raise ValueError("block_table and seq_lens need one row per request")
+    if o is not None:
+        _need(o, "o", o_dtype or dt, 3, (B, Hq, d))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2, (B, Hq))
+    _on_cuda(q=q, k_pages=k_pages, v_pages=v_pages, block_table=block_table, seq_lens=seq_lens,
+             o=o, lse=lse)
     return B, Hq, Hkv, d, num_pages, page_size, block_table.shape[1]
 
 
@@ -262,10 +292,7 @@ def fa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits: int,
     stream-ordered scratch).
     """
     B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
-        q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16)
-    _need(o, "o", torch.bfloat16, 3)
-    if lse is not None:
-        _need(lse, "lse", torch.float32, 2)
+        q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16, o, lse)
     ws_bytes = 0
     if workspace is not None:
         if not workspace.is_cuda or not workspace.is_contiguous():
@@ -287,10 +314,7 @@ def fa_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, num_spli
     different streams share the array and must not overlap.
     """
     B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
-        q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16)
-    _need(o, "o", torch.bfloat16, 3)
-    if lse is not None:
-        _need(lse, "lse", torch.float32, 2)
+        q, k_pages, v_pages, block_table, seq_lens, torch.bfloat16, o, lse)
     _check(load_library().fa_decode_paged_noalloc(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), page_size,
         int(num_splits), _ptr(o), _stream(stream), B, Hq, Hkv, d, max_blocks, num_pages,
@@ -326,6 +350,33 @@ def decode_paged_f32(q, k_pages, v_pages, block_table, seq_lens, scale: float = 
     return o, lse
 
 
+MATH_EXP2_FMA, MATH_EXP2_MUFU, MATH_SOFTCAP_LOG2 = 0, 1, 2
+
+
+def selftest_math(op: int, x: torch.Tensor, a: float = 0.0, b: float = 0.0, stream=None):
+    """Calls ``fa_selftest_math``: y = f(x) elementwise on the GPU for one of
+    the scalar functions of the prefill softmax (x: fp32 CUDA tensor)."""
+    _need(x, "x", torch.float32, x.dim())
+    _on_cuda(x=x)
+    y = torch.empty_like(x)
+    _check(load_library().fa_selftest_math(int(op), _ptr(x), _ptr(y), x.numel(), float(a),
+                                           float(b), _stream(stream)), "fa_selftest_math")
+    return y
+
+
+STALL_NONE, STALL_PREFILL, STALL_DECODE = 0, 1, 2
+
+
+def selftest_inject_stall(which: int, wait_limit_ns: int = 0) -> None:
+    """Calls ``fa_selftest_inject_stall`` (timeout-path tests only): makes one
+    warp of CTA 0 of the prefill (STALL_PREFILL) or decode (STALL_DECODE)
+    kernels wait on a barrier nothing arrives at, with the abortable-wait
+    limit set to wait_limit_ns (0 = the default 2 s).  (STALL_NONE, 0)
+    restores normal operation."""
+    _check(load_library().fa_selftest_inject_stall(int(which), int(wait_limit_ns)),
+           "fa_selftest_inject_stall")
+
+
 def device_error(stream=None) -> int:
     """Reads and clears the device error word (synchronises the stream)."""
     code = ctypes.c_int(0)
@@ -350,20 +401,17 @@ def fa_decode_paged_append(q, k_new, v_new, k_pages, v_pages, block_table, cache
     tables are given) into the page pool at cache_seqlens, then attends.
     k_pages / v_pages are modified in place; cache_seqlens is not."""
     B, Hq, Hkv, d, num_pages, page_size, max_blocks = _decode_shapes(
-        q, k_pages, v_pages, block_table, cache_seqlens, torch.bfloat16)
+        q, k_pages, v_pages, block_table, cache_seqlens, torch.bfloat16, o, lse)
     for t, n in ((k_new, "k_new"), (v_new, "v_new")):
-        _need(t, n, torch.bfloat16, 3)
-        if tuple(t.shape) != (B, Hkv, d):
-            raise ValueError(f"{n} must be [B, Hkv, d]")
-    _need(o, "o", torch.bfloat16, 3)
-    if lse is not None:
-        _need(lse, "lse", torch.float32, 2)
+        _need(t, n, torch.bfloat16, 3, (B, Hkv, d))
+    _on_cuda(k_new=k_new, v_new=v_new)
     max_pos, rd = 0, 0
     if (rotary_cos is None) != (rotary_sin is None):
         raise ValueError("give both rotary_cos and rotary_sin, or neither")
     if rotary_cos is not None:
         _need(rotary_cos, "rotary_cos", torch.float32, 2)
         _need(rotary_sin, "rotary_sin", torch.float32, 2)
+        _on_cuda(rotary_cos=rotary_cos, rotary_sin=rotary_sin)
         if rotary_sin.shape != rotary_cos.shape:
             raise ValueError("rotary_cos and rotary_sin shapes differ")
         max_pos = rotary_cos.shape[0]

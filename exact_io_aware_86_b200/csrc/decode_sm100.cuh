@@ -6,32 +6,43 @@
 // block_table[batch, max_blocks] and cache_seqlens; FlashDecoding / Split-KV
 // appendix: besides batch and heads, the KV length is split so several
 // thread blocks take different KV ranges of one head, followed by a final
-// reduce; "gsyq.cn FA vs FIA" section 2: the decode kernel walks the whole
-// KV cache block by block and lets the online softmax do the reduction, on
-// non-contiguous pages without copying them into a contiguous tensor):
+// reduce; GQA/MQA appendix: many query heads share one kv head; "gsyq.cn FA
+// vs FIA" section 2: the decode kernel walks the whole KV cache block by
+// block and lets the online softmax do the reduction, on non-contiguous
+// pages without copying them into a contiguous tensor):
 //
-//   Plan: a one-CTA kernel counts each request's page ranges (device-side
-//   seq_lens) and writes their prefix sums, so the split kernel can walk a
-//   flat list of non-empty ranges (the pages' Plan-Run split of scheduling
-//   and execution, "gsyq.cn FA vs FIA" section 2).
+//   Plan: each request's context is cut into page ranges; the exclusive
+//   prefix sums of the per-request range counts (from the device-side
+//   seq_lens) turn the ranges of all requests into one flat list of work
+//   items (the pages' Plan-Run split of scheduling and execution, "gsyq.cn
+//   FA vs FIA" section 2).  Every CTA of the split kernel builds the prefix
+//   itself in shared memory (up to PLAN_MAX_B requests); larger batches get
+//   it from a one-CTA plan kernel.
 //
-//   D1 (split kernel): persistent, one CTA per SM; CTA c takes ranges c,
-//   c + #CTAs, ... of the flat list (each for a group of up to 8 kv heads).
-//   A producer warp gathers each range's pages 16 tokens at a time
-//   into a shared-memory ring with TMA (3-D tensor maps over the pool with
-//   128-byte swizzle, one 16-token box of all the CTA's kv heads per 64-wide
-//   half of head_dim; page_size is a multiple of 16).  Each consumer warp owns one kv head and the Hq/Hkv <= 8 query
-//   heads that read it, so every K/V byte is read from HBM once for the whole
-//   group.  Scores and the P V product use warp-level bf16 tensor-core MMAs
-//   (S^T = K Q^T with tokens as rows, O^T += V^T P^T); the online softmax
-//   keeps a running max and sum per query head.  A range writes its
-//   normalised partial O and its LSE (fp32) to the workspace, or, when it is
-//   its request's only range, the final bf16 O and LSE directly.  In the
-//   automatic mode every range spans the same number of pages, so the flat
-//   list is made of near-equal items and the CTAs finish together.
+//   D1 (split kernel): persistent, one CTA per SM; CTA c takes items c,
+//   c + #CTAs, ... of the flat list.  An item is (request, page range, group
+//   of hpb kv heads, chunk of query heads).  A producer warp gathers the
+//   range's pages 16 tokens at a time into a shared-memory ring: with TMA
+//   (3-D tensor maps over the pool, 128-byte swizzle, one 16-token box of
+//   all the CTA's kv heads per 64-wide half of head_dim) when page_size is a
+//   multiple of 16, and otherwise token by token with 16-byte cp.async
+//   copies into the same swizzled layout (a stage may then span pages).
+//   Each consumer warp owns one kv head and one tile of 8 of the query heads
+//   that read it; all the warps of a kv head read the same shared-memory
+//   stage, so every K/V byte is read from HBM once for the whole group (a
+//   group of more than 64 query heads, 8 tiles, is split into chunks that
+//   each read it once).  Scores and the P V product use warp-level bf16
+//   tensor-core MMAs (S^T = K Q^T with tokens as rows, O^T += V^T P^T); the
+//   online softmax keeps a running max and sum per query head.  A range
+//   writes its normalised partial O and its LSE (fp32) to the workspace, or,
+//   when it is its request's only range, the final bf16 O and LSE directly.
+//   In the automatic mode every range spans the same number of pages, so
+//   the flat list is made of near-equal items and the CTAs finish together.
 //
 //   D2 (combine): per (request, query head), LSE = log sum_s exp(lse_s) and
-//   O = sum_s exp(lse_s - LSE) O_s over the request's ranges.
+//   O = sum_s exp(lse_s - LSE) O_s over the request's ranges.  It is
+//   launched as a programmatic dependent of D1: its CTAs are scheduled while
+//   D1 drains and wait (griddepcontrol.wait) until D1 has completed.
 #pragma once
 
 #include "ptx.cuh"
@@ -39,27 +50,51 @@
 namespace fa {
 namespace decode {
 
-constexpr int TOK = 16;      // tokens per pipeline stage (one MMA row block)
-constexpr int MAX_HPB = 8;   // kv heads per CTA
-constexpr int STAGES = 3;
-constexpr int MAX_GROUP = 8; // query heads per kv head (MMA N = 8)
+constexpr int TOK = 16;           // tokens per pipeline stage (one MMA row block)
+constexpr int QTILE = 8;          // query heads per consumer warp (MMA N = 8)
+constexpr int MAX_CONSUMERS = 8;  // consumer warps per CTA (kv heads x query tiles)
+constexpr int MAX_HPB = 8;        // kv heads per CTA
+constexpr int MAX_STAGES = 12;
+constexpr int STAGE_BUDGET = 192 * 1024;  // shared memory of the stage ring
+constexpr int PLAN_MAX_B = 2048;          // largest batch whose plan a CTA builds itself
+constexpr int SMEM_LIMIT = 232448;        // dynamic shared memory per CTA on sm_100
 
 struct Params {
-  const __nv_bfloat16* q;     // [B, Hq, D]
-  const int32_t* block_table; // [B, max_blocks]
-  const int32_t* seq_lens;    // [B]
-  const int32_t* split_prefix;  // [B+1] exclusive prefix of per-request range counts, or null
-  float* o_part;              // [B, Hq, s_max, D]   partial outputs (normalised)
-  float* lse_part;            // [B, Hq, s_max]      partial LSEs
-  __nv_bfloat16* o;           // [B, Hq, D]
-  float* lse;                 // [B, Hq] or null
-  int B, Hq, Hkv, group, hpb, ngroups;
+  const __nv_bfloat16* q;        // [B, Hq, D]
+  const __nv_bfloat16* k_pages;  // [num_pages, page_size, Hkv, D] (cp.async gather)
+  const __nv_bfloat16* v_pages;
+  const int32_t* block_table;    // [B, max_blocks]
+  const int32_t* seq_lens;       // [B]
+  const int32_t* split_prefix;   // [B+1] prefix from the plan kernel, or null
+  float* o_part;                 // [B, Hq, s_max, D]   partial outputs (normalised)
+  float* lse_part;               // [B, Hq, s_max]      partial LSEs
+  __nv_bfloat16* o;              // [B, Hq, D]
+  float* lse;                    // [B, Hq] or null
+  int B, Hq, Hkv, group;
+  int hpb;      // kv heads per CTA
+  int qpw;      // query tiles of 8 heads per kv head in a CTA (consumers = hpb * qpw)
+  int nq;       // chunks of qpw query tiles per kv head (items per range and kv-head group)
+  int ngroups;  // Hkv / hpb
   int page_size, max_blocks, num_pages;
-  int s_max;        // partial slots per (request, head)
+  int s_max;        // partial slots per (request, head); 1 = no split, no plan
   int chunk_pages;  // > 0: every range spans chunk_pages pages; 0: s_max near-equal ranges per request
   int half_bytes;   // bytes of the K (or V) part of one stage
+  int stages;       // ring length (<= MAX_STAGES)
+  int tma_gather;   // 1: TMA boxes (page_size % 16 == 0); 0: per-token cp.async copies
+  int local_plan;   // 1: each CTA builds the range prefix in shared memory
   float scale_log2;
 };
+
+// Shared memory of the split kernel after the ring: full and empty
+// barriers, the abort flag (16 bytes), the scan scratch of the plan (one int
+// per warp, 64 bytes), then the local plan (B + 1 ints).
+constexpr int RING_TAIL_BYTES = 2 * MAX_STAGES * 8 + 16 + 64;
+
+// Shared-memory bytes of the split kernel for these parameters, 1024-byte
+// alignment slack included.
+__host__ __device__ inline int split_smem_bytes(const Params& p) {
+  return p.stages * 2 * p.half_bytes + RING_TAIL_BYTES + (p.local_plan ? (p.B + 1) * 4 : 0) + 1024;
+}
 
 template <int D>
 struct Cfg {
@@ -150,12 +185,53 @@ __global__ void __launch_bounds__(1024) plan_kernel(const Params p, int32_t* __r
   if (tid == 0) prefix[p.B] = carry;
 }
 
-// Work item i -> (request b, range s, kv-head group y); items are the
-// non-empty ranges of every request, kv-head groups fastest.
-__device__ __forceinline__ void item_of(const Params& p, int i, int& b, int& s, int& y) {
-  y = i % p.ngroups;
-  const int bs = i / p.ngroups;
-  if (!p.split_prefix) {
+// Exclusive prefix sums of the per-request range counts into prefix[0..B]
+// (shared memory), by the whole CTA in chunks of blockDim.x requests.
+// `scratch` holds one int per warp.  Bad lengths are reported here.
+__device__ void build_plan(const Params& p, int* prefix, int* scratch) {
+  const int nthr = blockDim.x, tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  const int nwarps = nthr >> 5;
+  int carry = 0;
+  for (int base = 0; base < p.B; base += nthr) {
+    const int b = base + tid;
+    int n = 0;
+    if (b < p.B) {
+      int seq;
+      n = num_ranges(p, request_pages(p, b, seq, true));
+    }
+    int x = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int v = scratch[w];
+      before += w < warp ? v : 0;
+      total += v;
+    }
+    if (b < p.B) prefix[b] = carry + before + x - n;
+    carry += total;
+    __syncthreads();
+  }
+  if (tid == 0) prefix[p.B] = carry;
+  __syncthreads();
+}
+
+// Work item i -> (request b, range s, kv-head group g, query chunk qc);
+// items are the non-empty ranges of every request (all requests, one range
+// each, without a plan), kv-head groups and query chunks fastest.
+__device__ __forceinline__ void item_of(const Params& p, const int32_t* prefix, int i, int& b,
+                                        int& s, int& g, int& qc) {
+  const int per = p.ngroups * p.nq;
+  const int y = i % per;
+  g = y / p.nq;
+  qc = y - g * p.nq;
+  const int bs = i / per;
+  if (!prefix) {
     b = bs;
     s = 0;
     return;
@@ -163,19 +239,19 @@ __device__ __forceinline__ void item_of(const Params& p, int i, int& b, int& s, 
   int lo = 0, hi = p.B - 1;  // last b with prefix[b] <= bs
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(p.split_prefix + mid) <= bs) lo = mid; else hi = mid - 1;
+    if (prefix[mid] <= bs) lo = mid; else hi = mid - 1;
   }
   b = lo;
-  s = bs - __ldg(p.split_prefix + lo);
+  s = bs - prefix[lo];
 }
 
 // Token range [tok_begin, tok_end) of range s of request b.
-__device__ __forceinline__ void item_tokens(const Params& p, int b, int s, int& tok_begin,
-                                            int& tok_end, int& nranges) {
+__device__ __forceinline__ void item_tokens(const Params& p, bool planned, int b, int s,
+                                            int& tok_begin, int& tok_end, int& nranges) {
   int seq;
-  // the plan kernel reports bad lengths when there is a plan; otherwise here
-  const int npages = request_pages(p, b, seq, !p.split_prefix);
-  if (!p.split_prefix) {
+  // with a plan, bad lengths were reported while building it; otherwise here
+  const int npages = request_pages(p, b, seq, !planned);
+  if (!planned) {
     tok_begin = 0;
     tok_end = seq;
     nranges = 1;
@@ -188,10 +264,24 @@ __device__ __forceinline__ void item_tokens(const Params& p, int b, int s, int& 
   nranges = num_ranges(p, npages);
 }
 
-// Persistent: CTA c takes items c, c + gridDim.x, ...; the TMA ring runs on
+// 16-byte global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros
+// and reads nothing.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// Arrives on the mbarrier once every cp.async this thread issued so far has
+// completed (the arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Persistent: CTA c takes items c, c + gridDim.x, ...; the ring runs on
 // across item boundaries.
 template <int D>
-__global__ void __launch_bounds__((MAX_HPB + 1) * 32)
+__global__ void __launch_bounds__((MAX_CONSUMERS + 1) * 32, 1)
     split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const Params p) {
   using C = Cfg<D>;
@@ -199,32 +289,53 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int sbytes = stage_bytes(p.half_bytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * sbytes);
-  uint64_t* empty = full + STAGES;
-  int* abort_flag = reinterpret_cast<int*>(empty + STAGES);
+  const int nstages = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + nstages * sbytes);
+  uint64_t* empty = full + MAX_STAGES;
+  int* abort_flag = reinterpret_cast<int*>(empty + MAX_STAGES);
+  uint64_t* stall_bar = reinterpret_cast<uint64_t*>(abort_flag + 2);  // timeout test hook
+  int* scan_scratch = abort_flag + 4;  // one int per warp, only while the plan is built
+  int32_t* local_prefix = abort_flag + 4 + 16;
   volatile int* abort = abort_flag;
 
   const int warp = warp_id(), lane = lane_id();
-  const int nconsumers = p.hpb;
+  const int nconsumers = p.hpb * p.qpw;
+
+  // the combine kernel (a programmatic dependent) may be scheduled now; it
+  // waits for this grid to complete before it reads anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+    for (int s = 0; s < nstages; ++s) {
+      // TMA: one arrive.expect_tx per stage; cp.async: one arrival per producer lane
+      mbar_init(&full[s], p.tma_gather ? 1 : 32);
       mbar_init(&empty[s], nconsumers);
     }
     *abort_flag = 0;
+    mbar_init(stall_bar, 1);  // never arrived at
     fence_mbar_init();
   }
+  const int32_t* prefix = nullptr;
+  if (p.s_max > 1) {
+    if (p.local_plan) {
+      build_plan(p, local_prefix, scan_scratch);
+      prefix = local_prefix;
+    } else {
+      prefix = p.split_prefix;
+    }
+  }
   __syncthreads();
-
-  const int total = (p.split_prefix ? __ldg(p.split_prefix + p.B) : p.B) * p.ngroups;
+  const bool planned = prefix != nullptr;
+  const int total = (planned ? prefix[p.B] : p.B) * p.ngroups * p.nq;
 
   if (warp == nconsumers) {
     // ======================= producer (converged warp) =======================
     // The whole warp runs the loop: the block-table entries of 32 stages are
-    // fetched at once, one per lane, and broadcast by shuffle, so no stage
-    // waits on a dependent global load; one elected lane issues the copies.
-    if (lane == 0) {
+    // fetched at once, one per lane, and broadcast by shuffle (TMA gather), or
+    // each of 16 lanes looks up its token's page (cp.async gather), so no
+    // stage waits on a dependent global load; TMA copies are issued by one
+    // elected lane, cp.async copies by all lanes.
+    if (lane == 0 && p.tma_gather) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
@@ -232,67 +343,109 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
     int g = 0;  // stages issued so far (ring position)
     bool ok = true;
     for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-      int b, s, y, tb, te, nr;
-      item_of(p, i, b, s, y);
-      item_tokens(p, b, s, tb, te, nr);
-      const int kvh0 = y * p.hpb;
+      int b, s, grp, qc, tb, te, nr;
+      item_of(p, prefix, i, b, s, grp, qc);
+      item_tokens(p, planned, b, s, tb, te, nr);
+      const int kvh0 = grp * p.hpb;
       const int32_t* bt = p.block_table + (size_t)b * p.max_blocks;
       const int nst = te > tb ? (te - tb + TOK - 1) / TOK : 0;
       int page_of_lane = 0;
       for (int st = 0; st < nst; ++st, ++g) {
-        if ((st & 31) == 0) {
-          const int sl = st + lane;  // the stage whose page this lane looks up
-          page_of_lane = sl < nst ? __ldg(bt + (tb + sl * TOK) / p.page_size) : 0;
-        }
-        const int page = __shfl_sync(0xffffffffu, page_of_lane, st & 31);
-        const int slot = g % STAGES;
-        if (!mbar_wait(&empty[slot], ((g / STAGES) & 1) ^ 1, abort)) { ok = false; break; }
-        // page_size is a multiple of TOK, so a stage never crosses a page
+        const int slot = g % nstages;
         const int t0 = tb + st * TOK;
-        int z;
-        if (page < 0 || page >= p.num_pages) {
-          if (lane == 0) report_error(kDevErrBounds);
-          z = -TOK;  // whole box outside the pool: TMA fills zeros
-        } else {
-          z = page * p.page_size + (t0 % p.page_size);
-        }
-        expect_tx_el(&full[slot], 2 * p.half_bytes);
         uint8_t* kdst = smem + slot * sbytes;
         uint8_t* vdst = kdst + p.half_bytes;
-        // one box per 64-wide half of head_dim holds all the CTA's kv heads
-        for (int pn = 0; pn < C::PANELS; ++pn) {
-          const int off = pn * p.hpb * BOX_BYTES;
-          tma_load_3d_el(kdst + off, &tmK, &full[slot], pn * 64, z, kvh0);
-          tma_load_3d_el(vdst + off, &tmV, &full[slot], pn * 64, z, kvh0);
+        if (p.tma_gather) {
+          if ((st & 31) == 0) {
+            const int sl = st + lane;  // the stage whose page this lane looks up
+            page_of_lane = sl < nst ? __ldg(bt + (tb + sl * TOK) / p.page_size) : 0;
+          }
+          const int page = __shfl_sync(0xffffffffu, page_of_lane, st & 31);
+          if (!mbar_wait(&empty[slot], ((g / nstages) & 1) ^ 1, abort)) { ok = false; break; }
+          // page_size is a multiple of TOK, so a stage never crosses a page
+          int z;
+          if (page < 0 || page >= p.num_pages) {
+            if (lane == 0) report_error(kDevErrBounds);
+            z = -TOK;  // whole box outside the pool: TMA fills zeros
+          } else {
+            z = page * p.page_size + (t0 % p.page_size);
+          }
+          expect_tx_el(&full[slot], 2 * p.half_bytes);
+          // one box per 64-wide half of head_dim holds all the CTA's kv heads
+          for (int pn = 0; pn < C::PANELS; ++pn) {
+            const int off = pn * p.hpb * BOX_BYTES;
+            tma_load_3d_el(kdst + off, &tmK, &full[slot], pn * 64, z, kvh0);
+            tma_load_3d_el(vdst + off, &tmV, &full[slot], pn * 64, z, kvh0);
+          }
+        } else {
+          // token `lane` (< 16) of this stage: its page, or -1 (past the
+          // range, or a bad entry: its rows are filled with zeros)
+          const int valid = min(TOK, te - t0);
+          int pg = -1;
+          if (lane < valid) {
+            pg = __ldg(bt + (t0 + lane) / p.page_size);
+            if (pg < 0 || pg >= p.num_pages) {
+              report_error(kDevErrBounds);
+              pg = -1;
+            }
+          }
+          if (!mbar_wait(&empty[slot], ((g / nstages) & 1) ^ 1, abort)) { ok = false; break; }
+          // 16-byte chunks of the stage's (token, kv head) rows, consecutive
+          // lanes on consecutive chunks of a row: a row of one token's kv
+          // heads is contiguous in the pool
+          constexpr int CPR = D / 8;  // chunks per row
+          const uint32_t kbase = smem_u32(kdst), vbase = smem_u32(vdst);
+          for (int q = lane; q < TOK * p.hpb * CPR; q += 32) {
+            const int row = q / CPR, c16 = q - row * CPR;
+            const int tok = row / p.hpb, hh = row - tok * p.hpb;
+            const int page = __shfl_sync(0xffffffffu, pg, tok);
+            const uint32_t dst = kv_off(p.hpb, c16 >> 3, hh, tok, c16 & 7);
+            size_t src = 0;
+            uint32_t bytes = 0;
+            if (page >= 0) {
+              const int pos = page * p.page_size + (t0 + tok) % p.page_size;
+              src = ((size_t)pos * p.Hkv + kvh0 + hh) * D + c16 * 8;
+              bytes = 16;
+            }
+            cp_async_16(kbase + dst, p.k_pages + src, bytes);
+            cp_async_16(vbase + dst, p.v_pages + src, bytes);
+          }
+          cp_async_arrive_noinc(&full[slot]);
         }
       }
     }
     // every load issued must land before the CTA exits
-    for (int s = 0; s < STAGES && s < g; ++s) {
-      const int last = g - 1 - ((g - 1 - s) % STAGES);
-      mbar_wait_bounded(&full[last % STAGES], (last / STAGES) & 1);
+    for (int s = 0; s < nstages && s < g; ++s) {
+      const int last = g - 1 - ((g - 1 - s) % nstages);
+      mbar_wait_bounded(&full[last % nstages], (last / nstages) & 1);
     }
-  } else {
-    // ======================= consumers: one warp per kv head =======================
-    const int hh = warp;
+  } else if (warp < nconsumers) {
+    // ============ consumers: one warp per (kv head, tile of 8 query heads) ============
+    const int hh = warp / p.qpw;   // kv head of the CTA's group
+    const int qtw = warp % p.qpw;  // query tile within the chunk
     const int g8 = lane >> 2, tq = lane & 3;
     const float sl = p.scale_log2;
     const uint32_t sbase = smem_u32(smem);
     const int lm = lane >> 3, lr = lane & 7;  // ldmatrix row/chunk assignment of this lane
     int g = 0;  // stages consumed so far (ring position)
     bool ok = true;
+    // timeout test hook: this warp's first stage wait is on a barrier that
+    // nothing arrives at
+    bool stall = warp == 0 && blockIdx.x == 0 &&
+                 *reinterpret_cast<volatile int*>(&g_stall_test) == kStallDecode;
     for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-      int b, s, y, tb, te, nr;
-      item_of(p, i, b, s, y);
-      item_tokens(p, b, s, tb, te, nr);
-      const int kvh = y * p.hpb + hh;
+      int b, s, grp, qc, tb, te, nr;
+      item_of(p, prefix, i, b, s, grp, qc);
+      item_tokens(p, planned, b, s, tb, te, nr);
+      const int kvh = grp * p.hpb + hh;
+      const int qt = qc * p.qpw + qtw;  // query tile: heads qt*8 .. qt*8+7 of the kv head's group
       const int nst = te > tb ? (te - tb + TOK - 1) / TOK : 0;
-      // Q^T fragments (MMA B operand, k = head_dim, n = query head of the group)
+      // Q^T fragments (MMA B operand, k = head_dim, n = query head of the tile)
       uint32_t qb0[C::KS], qb1[C::KS];
       {
-        const bool real = g8 < p.group;
+        const bool real = qt * QTILE + g8 < p.group;
         const __nv_bfloat16* qrow =
-            p.q + ((size_t)b * p.Hq + (size_t)kvh * p.group + (real ? g8 : 0)) * D;
+            p.q + ((size_t)b * p.Hq + (size_t)kvh * p.group + qt * QTILE + (real ? g8 : 0)) * D;
 #pragma unroll
         for (int ks = 0; ks < C::KS; ++ks) {
           const uint32_t* w = reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * tq);
@@ -303,18 +456,25 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
       float acc[C::KS][4];
 #pragma unroll
       for (int mt = 0; mt < C::KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-      // query heads 2tq, 2tq+1: running max, exact sum of exp (for the LSE) and
-      // sum of the bf16-rounded weights the PV MMA uses (normalises O)
+      // query heads 2tq, 2tq+1 of the tile: running max, exact sum of exp (for
+      // the LSE) and sum of the bf16-rounded weights the PV MMA uses
+      // (normalises O)
       float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
       for (int st = 0; st < nst; ++st, ++g) {
-        const int slot = g % STAGES;
-        if (!mbar_wait(&full[slot], (g / STAGES) & 1, abort)) { ok = false; break; }
+        const int slot = g % nstages;
+        if (!mbar_wait(stall ? stall_bar : &full[slot], (g / nstages) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        stall = false;
         const uint32_t kb = sbase + slot * sbytes;
         const uint32_t vb = kb + p.half_bytes;
         const int valid = min(TOK, te - (tb + st * TOK));
-        if (valid < TOK) {
+        if (valid < TOK && p.tma_gather) {
           // V rows past the context are not part of the sum; their P is zero,
-          // but 0 * (garbage) may be NaN, so clear them for this warp's head.
+          // but 0 * (garbage) may be NaN, so clear them for this warp's head
+          // (every warp of the head writes the same zeros before its reads;
+          // the cp.async gather already filled them with zeros).
           uint8_t* vgen = smem + slot * sbytes + p.half_bytes;
           for (int idx = lane; idx < (TOK - valid) * C::PANELS * 8; idx += 32) {
             const int tok = valid + idx / (C::PANELS * 8);
@@ -377,7 +537,7 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
           ldmatrix_x4_trans(vb + kv_off(p.hpb, d0 >> 6, hh, tok, (d0 & 63) >> 3), a0, a1, a2, a3);
           mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
         }
-        if (valid < TOK) fence_proxy_async_smem();
+        if (valid < TOK && p.tma_gather) fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
       }
@@ -394,7 +554,8 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
       const float ln2 = 0.69314718055994531f;
       const float lse0 = l0 > 0.f ? (m0 + __log2f(l0)) * ln2 : -INFINITY;
       const float lse1 = l1 > 0.f ? (m1 + __log2f(l1)) * ln2 : -INFINITY;
-      const int n0 = 2 * tq, n1 = 2 * tq + 1;
+      // heads of the tile held by this lane, as indices in the kv head's group
+      const int n0 = qt * QTILE + 2 * tq, n1 = n0 + 1;
       const size_t head0 = (size_t)b * p.Hq + (size_t)kvh * p.group;
       if (nr > 1) {
         const int S = p.s_max;
@@ -451,17 +612,23 @@ __global__ void __launch_bounds__((MAX_HPB + 1) * 32)
 constexpr int COMBINE_WARPS = 8;
 
 template <int D>
-__global__ void __launch_bounds__(COMBINE_WARPS * 32)
-    combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                   const int32_t* __restrict__ prefix, __nv_bfloat16* __restrict__ o,
-                   float* __restrict__ lse, int Hq, int S) {
+__global__ void __launch_bounds__(COMBINE_WARPS * 32) combine_kernel(const Params p) {
   constexpr int PER = D / 32;  // output elements per lane
   __shared__ float red[COMBINE_WARPS][D];
   __shared__ float wred[COMBINE_WARPS];
+  // launched as a programmatic dependent of the split kernel: wait until it
+  // has completed and its partial results are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float* __restrict__ o_part = p.o_part;
+  const float* __restrict__ lse_part = p.lse_part;
+  __nv_bfloat16* __restrict__ o = p.o;
+  float* __restrict__ lse = p.lse;
+  const int Hq = p.Hq, S = p.s_max;
   const int r = blockIdx.x;
   const int b = r / Hq;
   const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
-  const int n = __ldg(prefix + b + 1) - __ldg(prefix + b);
+  int seq;
+  const int n = num_ranges(p, request_pages(p, b, seq, false));
   if (n == 1) return;
   const float* lp = lse_part + (size_t)r * S;
   const float log2e = 1.4426950408889634f;

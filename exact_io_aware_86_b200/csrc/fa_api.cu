@@ -74,19 +74,69 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / sqrtf((float)d); }
 
-// Largest divisor of Hkv that is <= 8: kv heads handled by one decode CTA.
-int heads_per_cta(int Hkv) {
-  for (int h = fa::decode::MAX_HPB; h >= 1; --h)
-    if (Hkv % h == 0) return h;
-  return 1;
+// max_seqlen <= 0 means "not given": every sequence is at most T long, and
+// the work list can hold MAX_LEVELS * 256 rows per sequence.
+int resolve_max_seqlen(int max_seqlen, int total_tokens) {
+  if (max_seqlen > 0) return max_seqlen;
+  return std::min<long long>(total_tokens,
+                             (long long)fa::prefill::MAX_LEVELS * fa::prefill::ROWS_PER_ITEM);
+}
+
+// How the decode spreads the heads over a CTA's consumer warps: each warp
+// takes one kv head and one tile of 8 of its Hq / Hkv query heads.  A CTA
+// holds hpb kv heads (a divisor of Hkv) with qpw query tiles each, at most 8
+// warps; a kv head with more than 8 tiles (more than 64 query heads) is
+// split into nq chunks of 8 tiles, which are separate work items.
+struct DecodeLayout {
+  int hpb, qpw, nq;
+};
+
+DecodeLayout decode_layout(int Hq, int Hkv) {
+  using namespace fa::decode;
+  const int tiles = (Hq / Hkv + QTILE - 1) / QTILE;
+  DecodeLayout L{1, tiles, 1};
+  if (tiles > MAX_CONSUMERS) {
+    L.qpw = MAX_CONSUMERS;
+    L.nq = (tiles + MAX_CONSUMERS - 1) / MAX_CONSUMERS;
+    return L;
+  }
+  for (int h = std::min(MAX_HPB, MAX_CONSUMERS / tiles); h >= 1; --h)
+    if (Hkv % h == 0) {
+      L.hpb = h;
+      break;
+    }
+  return L;
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+constexpr int kMaxDevices = 64;
+
+// Launch set-up of one kernel: the dynamic shared-memory limit is an
+// attribute of the kernel on a device, so it is set once per device (under a
+// lock, as several host threads may launch on several devices), together
+// with the register count the compiled kernel launches with.
+struct KernelSetup {
+  std::mutex mu;
+  int state[kMaxDevices] = {};  // 0 not yet, 1 ready, -1 failed
+  int regs[kMaxDevices] = {};
+};
+
 template <typename K>
-bool set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-         cudaSuccess;
+bool setup_kernel(KernelSetup& ks, K kernel, int smem_bytes, int* regs = nullptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(ks.mu);
+  if (ks.state[dev] == 0) {
+    cudaFuncAttributes a;
+    const bool ok = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem_bytes) == cudaSuccess &&
+                    cudaFuncGetAttributes(&a, kernel) == cudaSuccess;
+    ks.regs[dev] = ok ? a.numRegs : 0;
+    ks.state[dev] = ok ? 1 : -1;
+  }
+  if (regs) *regs = ks.regs[dev];
+  return ks.state[dev] == 1;
 }
 
 // Mask variants after normalisation: window bounds -1 (no limit) or in
@@ -107,16 +157,12 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
                          float qk_descale = 1.f, float v_descale = 1.f) {
   using namespace fa::prefill;
   using C = Cfg<D, FP8>;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   const cuuint32_t box[2] = {(cuuint32_t)C::PANEL_ELEMS, (cuuint32_t)BM};  // 128 B x 128 rows
   {
     const cuuint64_t dims[2] = {(cuuint64_t)Hq * D, (cuuint64_t)T};
     const cuuint64_t str[1] = {(cuuint64_t)Hq * D * C::ESIZE};
     if (!make_map(&tq, q, 2, dims, str, box, FP8)) return FA_ERR_CUDA;
-    // O is bf16 whatever the input type: 64-column x 128-row store boxes
-    const cuuint64_t ostr[1] = {(cuuint64_t)Hq * D * 2};
-    const cuuint32_t obox[2] = {64, (cuuint32_t)BM};
-    if (!make_map(&to, o, 2, dims, ostr, obox)) return FA_ERR_CUDA;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)Hkv * D, (cuuint64_t)T};
@@ -153,17 +199,14 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   if (grid > 0x7fffffff) return FA_ERR_UNSUPPORTED;
 
   const int smem = smem_bytes<D, FP8>();
-  static bool attr_ok = set_smem(prefill_kernel<D, GENERAL, FP8>, smem);
-  if (!attr_ok) return FA_ERR_CUDA;
+  static KernelSetup setup;
+  int launch_regs = 0;
+  if (!setup_kernel(setup, prefill_kernel<D, GENERAL, FP8>, smem, &launch_regs)) return FA_ERR_CUDA;
   // The kernel hands registers between its warpgroups with setmaxnreg; the
   // split only fits if the launch allots kRegsLaunch registers per thread
   // (otherwise setmaxnreg.inc could never be satisfied).
-  static int launch_regs = [] {
-    cudaFuncAttributes a;
-    return cudaFuncGetAttributes(&a, prefill_kernel<D, GENERAL, FP8>) == cudaSuccess ? a.numRegs : -1;
-  }();
   if (launch_regs < (int)kRegsLaunch) return FA_ERR_UNSUPPORTED;
-  prefill_kernel<D, GENERAL, FP8><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, to, p);
+  prefill_kernel<D, GENERAL, FP8><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -176,8 +219,9 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 // (1 - the partial-output traffic relative to the K/V bytes - a fixed
 // per-range cost), with ranges of at least 256 tokens.
 int auto_chunk_pages(int B, int Hq, int Hkv, int max_blocks, int page_size, int num_sms) {
-  const int hpb = heads_per_cta(Hkv);
-  const long long ngroups = Hkv / hpb;
+  const DecodeLayout L = decode_layout(Hq, Hkv);
+  const int hpb = L.hpb;
+  const long long ngroups = (long long)(Hkv / hpb) * L.nq;  // items per range
   const int G = num_sms > 0 ? num_sms : 148;
   const long long U = (long long)B * max_blocks * ngroups;
   const int c_min = std::min(max_blocks, std::max(1, ceil_div(256, page_size)));
@@ -216,30 +260,23 @@ fa_status launch_decode(const void* q, const void* kp, const void* vp, const int
                         cudaStream_t stream, int B, int Hq, int Hkv, int max_blocks, int num_pages,
                         float scale, float* lse, void* ws) {
   using namespace fa::decode;
-  const int hpb = heads_per_cta(Hkv);
+  const DecodeLayout L = decode_layout(Hq, Hkv);
   const int sms = num_sms_current();
   if (sms <= 0) return FA_ERR_CUDA;
-  CUtensorMap tk, tv;
-  {
-    // dimensions (head_dim, token, kv head): a box of the CTA's heads lands in
-    // shared memory as [head][token][64 dims] (see decode_sm100.cuh)
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)num_pages * (cuuint64_t)page_size,
-                                (cuuint64_t)Hkv};
-    const cuuint64_t str[2] = {(cuuint64_t)Hkv * D * 2, (cuuint64_t)D * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)TOK, (cuuint32_t)hpb};
-    if (!make_map(&tk, kp, 3, dims, str, box)) return FA_ERR_CUDA;
-    if (!make_map(&tv, vp, 3, dims, str, box)) return FA_ERR_CUDA;
-  }
   Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_pages = static_cast<const __nv_bfloat16*>(kp);
+  p.v_pages = static_cast<const __nv_bfloat16*>(vp);
   p.block_table = bt;
   p.seq_lens = sl;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.group = Hq / Hkv;
-  p.hpb = hpb;
-  p.ngroups = Hkv / hpb;
+  p.hpb = L.hpb;
+  p.qpw = L.qpw;
+  p.nq = L.nq;
+  p.ngroups = Hkv / L.hpb;
   p.page_size = page_size;
   p.max_blocks = max_blocks;
   p.num_pages = num_pages;
@@ -250,34 +287,69 @@ fa_status launch_decode(const void* q, const void* kp, const void* vp, const int
     p.chunk_pages = 0;
     p.s_max = num_splits;
   }
-  p.half_bytes = Cfg<D>::PANELS * hpb * BOX_BYTES;
+  p.half_bytes = Cfg<D>::PANELS * L.hpb * BOX_BYTES;
+  p.stages = std::min(MAX_STAGES, STAGE_BUDGET / stage_bytes(p.half_bytes));
+  p.tma_gather = page_size % TOK == 0 ? 1 : 0;
   p.scale_log2 = resolve_scale(scale, D) * kLog2e;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   const bool split = p.s_max > 1;
+  p.local_plan = split && B <= PLAN_MAX_B ? 1 : 0;
   const size_t opart_bytes = round_up((size_t)B * Hq * p.s_max * D * sizeof(float), 256);
   const size_t lpart_bytes = round_up((size_t)B * Hq * p.s_max * sizeof(float), 256);
   p.o_part = split ? static_cast<float*>(ws) : nullptr;
   p.lse_part = split ? reinterpret_cast<float*>(static_cast<char*>(ws) + opart_bytes) : nullptr;
-  int32_t* prefix = split ? reinterpret_cast<int32_t*>(static_cast<char*>(ws) + opart_bytes + lpart_bytes)
-                          : nullptr;
+  int32_t* prefix = split && !p.local_plan
+                        ? reinterpret_cast<int32_t*>(static_cast<char*>(ws) + opart_bytes + lpart_bytes)
+                        : nullptr;
   p.split_prefix = prefix;
+  const long long items = (split ? (long long)B * p.s_max : (long long)B) * p.ngroups * p.nq;
+  if (items > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
 
-  if (split) {
+  CUtensorMap tk, tv;
+  std::memset(&tk, 0, sizeof(tk));
+  std::memset(&tv, 0, sizeof(tv));
+  if (p.tma_gather) {
+    // dimensions (head_dim, token, kv head): a box of the CTA's heads lands in
+    // shared memory as [head][token][64 dims] (see decode_sm100.cuh).  An
+    // empty pool is mapped as one page, which no copy reads (every page index
+    // is then out of range and fetched as zeros).
+    const cuuint64_t dims[3] = {(cuuint64_t)D,
+                                (cuuint64_t)std::max(num_pages, 1) * (cuuint64_t)page_size,
+                                (cuuint64_t)Hkv};
+    const cuuint64_t str[2] = {(cuuint64_t)Hkv * D * 2, (cuuint64_t)D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)TOK, (cuuint32_t)L.hpb};
+    if (!make_map(&tk, kp, 3, dims, str, box)) return FA_ERR_CUDA;
+    if (!make_map(&tv, vp, 3, dims, str, box)) return FA_ERR_CUDA;
+  }
+
+  if (prefix) {
     plan_kernel<<<1, 1024, 0, stream>>>(p, prefix);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  const int smem = STAGES * stage_bytes(p.half_bytes) + 1024 + 64;
-  static bool attr_ok = set_smem(split_kernel<D>, STAGES * stage_bytes(Cfg<D>::PANELS * MAX_HPB * BOX_BYTES) + 1024 + 64);
-  if (!attr_ok) return FA_ERR_CUDA;
-  const long long upper = (split ? (long long)B * p.s_max : (long long)B) * p.ngroups;
-  const int grid = (int)(upper < sms ? upper : sms);
-  split_kernel<D><<<grid, (hpb + 1) * 32, smem, stream>>>(tk, tv, p);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  if (split) {
-    combine_kernel<D><<<B * Hq, COMBINE_WARPS * 32, 0, stream>>>(p.o_part, p.lse_part, prefix,
-                                                                 p.o, lse, Hq, p.s_max);
+  static KernelSetup setup;
+  if (!setup_kernel(setup, split_kernel<D>, SMEM_LIMIT)) return FA_ERR_CUDA;
+  const int smem = split_smem_bytes(p);
+  const int grid = (int)std::min<long long>(items, sms);
+  if (grid > 0) {
+    split_kernel<D><<<grid, (L.hpb * L.qpw + 1) * 32, smem, stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (split) {
+    // a programmatic dependent of the split kernel: its CTAs are scheduled
+    // while the split kernel drains and wait for it to complete
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(B * Hq));
+    cfg.blockDim = dim3(COMBINE_WARPS * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = grid > 0 ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, combine_kernel<D>, p) != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
 }
@@ -292,12 +364,13 @@ fa_status fa_prefill_ex(const void* q, const void* k, const void* v, void* o, fl
                         int window_left, int window_right, float softcap,
                         const float* alibi_slopes, int alibi_batch_stride) {
   if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_INVALID_ARG;
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0 || max_seqlen < 0)
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0)
     return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(cu_seqlens, 4) || (lse && !aligned(lse, 4)) ||
       (alibi_slopes && !aligned(alibi_slopes, 4)))
     return FA_ERR_INVALID_ARG;
+  max_seqlen = resolve_max_seqlen(max_seqlen, total_tokens);
   if (!(softcap >= 0.f) || std::isinf(softcap) || alibi_batch_stride < 0)
     return FA_ERR_INVALID_ARG;
   Variant var;
@@ -332,11 +405,12 @@ fa_status fa_prefill_fp8(const void* q, const void* k, const void* v, void* o, f
                          float scale, float q_descale, float k_descale, float v_descale,
                          fa_stream_t stream, int total_tokens, int max_seqlen) {
   if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_INVALID_ARG;
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0 || max_seqlen < 0)
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || total_tokens < 0)
     return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(cu_seqlens, 4) || (lse && !aligned(lse, 4)))
     return FA_ERR_INVALID_ARG;
+  max_seqlen = resolve_max_seqlen(max_seqlen, total_tokens);
   for (float x : {q_descale, k_descale, v_descale})
     if (!(x > 0.f) || std::isinf(x)) return FA_ERR_INVALID_ARG;
   if (d != 128) return FA_ERR_UNSUPPORTED;
@@ -392,12 +466,10 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
       (workspace && !aligned(workspace, 256)))
     return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (Hq / Hkv > fa::decode::MAX_GROUP) return FA_ERR_UNSUPPORTED;
-  if (page_size % fa::decode::TOK != 0) return FA_ERR_UNSUPPORTED;
   if ((long long)num_pages * page_size > 0x7fffffffLL ||
       (long long)max_blocks_per_seq * page_size > 0x7fffffffLL)
     return FA_ERR_UNSUPPORTED;
-  if (B > 65535 || Hkv / heads_per_cta(Hkv) > 65535) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (B == 0) return FA_OK;
   const int S = num_splits == 0
                     ? fa_decode_auto_splits(B, Hq, Hkv, max_blocks_per_seq, page_size, 0)
@@ -455,12 +527,10 @@ fa_status fa_decode_paged_append(const void* q, const void* k_new, const void* v
     return FA_ERR_INVALID_ARG;
   // the attention step has the limits of fa_decode_paged
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (Hq / Hkv > fa::decode::MAX_GROUP) return FA_ERR_UNSUPPORTED;
-  if (page_size % fa::decode::TOK != 0) return FA_ERR_UNSUPPORTED;
   if ((long long)num_pages * page_size > 0x7fffffffLL ||
       (long long)max_blocks_per_seq * page_size > 0x7fffffffLL)
     return FA_ERR_UNSUPPORTED;
-  if (B > 65535 || Hkv / heads_per_cta(Hkv) > 65535) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (B == 0) return FA_OK;
   const int S = num_splits == 0
                     ? fa_decode_auto_splits(B, Hq, Hkv, max_blocks_per_seq, page_size, 0)
@@ -584,6 +654,58 @@ int fa_version(void) { return 100; }
 }  // extern "C"
 
 // --------------------------------------------------------------------------
+// Self-test hook: the scalar functions the prefill kernel computes the
+// softmax weights with, evaluated element by element on the GPU so a test
+// can compare them with an exact reference over their whole input range.
+// --------------------------------------------------------------------------
+namespace fa {
+namespace selftest {
+
+__global__ void math_kernel(int op, const float* __restrict__ x, float* __restrict__ y, int n,
+                            float a, float b) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  const float x0 = x[i], x1 = two ? x[i + 1] : 0.f;
+  float y0 = 0.f, y1 = 0.f;
+  if (op == FA_MATH_EXP2_FMA) {
+    f2_unpack(exp2_fma_pair(f2_pack(x0, x1)), y0, y1);
+  } else if (op == FA_MATH_EXP2_MUFU) {
+    y0 = ex2(x0);
+    y1 = ex2(x1);
+  } else {
+    y0 = softcap_log2(x0, a, b);
+    y1 = softcap_log2(x1, a, b);
+  }
+  y[i] = y0;
+  if (two) y[i + 1] = y1;
+}
+
+}  // namespace selftest
+}  // namespace fa
+
+extern "C" fa_status fa_selftest_inject_stall(int which, unsigned long long wait_limit_ns) {
+  if (which != 0 && which != FA_STALL_PREFILL && which != FA_STALL_DECODE) return FA_ERR_INVALID_ARG;
+  const unsigned long long limit = wait_limit_ns ? wait_limit_ns : fa::kWaitLimitNs;
+  if (cudaMemcpyToSymbol(fa::g_stall_test, &which, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(fa::g_wait_limit_ns, &limit, sizeof(limit)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+extern "C" fa_status fa_selftest_math(int op, const float* x, float* y, int n, float a, float b,
+                                      fa_stream_t stream) {
+  if (op != FA_MATH_EXP2_FMA && op != FA_MATH_EXP2_MUFU && op != FA_MATH_SOFTCAP_LOG2)
+    return FA_ERR_INVALID_ARG;
+  if (n < 0 || (n > 0 && (!x || !y)) || !aligned(x, 4) || !aligned(y, 4)) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  const int pairs = (n + 1) / 2;
+  fa::selftest::math_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      op, x, y, n, a, b);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// --------------------------------------------------------------------------
 // Paged decode without any allocation (fa_decode_paged_noalloc).
 //
 // Some callers cannot allocate device memory at the point where they run a
@@ -598,8 +720,6 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per device
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
-
-constexpr int kMaxDevices = 64;
 
 // Device address of g_decode_scratch on the current device.  The first call
 // on each device looks it up (cudaGetSymbolAddress with that device current)

@@ -11,8 +11,9 @@
 //   running row max m and sum l, write P = exp(S*scale - m) back into tensor
 //   memory as bf16, and the tensor cores accumulate O += P V_j in tensor
 //   memory.  At the end O / l is stored as bf16 and LSE = ln2*(m + log2 l).
-//   Full tiles of O leave through a swizzled shared-memory staging panel and
-//   TMA stores; a tile that runs past its sequence's end is stored row by row.
+//   O leaves through a small shared-memory staging region per warp, read
+//   back for coalesced 128-byte global stores (rows past a sequence end are
+//   skipped).
 //
 // CTA layout (384 threads = 3 warpgroups, one CTA per SM, persistent):
 //   warp 0      TMA producer: Q tiles once per work item (one barrier pair
@@ -45,11 +46,15 @@
 // the result is exact up to rounding.
 //
 // Softmax arithmetic per score: one three-input max per two scores, one
-// packed FMA per two scores for s*scale*log2e - m, 2^x on the MUFU unit for
-// three of every four pairs and on the FMA pipe (exp2_fma_pair) for the
-// fourth, which balances the two units.  P is rounded to bf16 for the MMA;
-// O is divided by the sum of those rounded values (so O is a weighted mean
-// with exactly the weights used) and the LSE uses the unrounded sum.
+// packed FMA per two scores for s*scale*log2e - m, 2^x on the MUFU unit
+// (POLY_EVERY > 0 moves one pair in POLY_EVERY to the FMA pipe,
+// exp2_fma_pair; measured, every instantiation is faster all on MUFU), one
+// packed add per two scores into the unrounded row sum and two mixed adds
+// into the sum of the bf16-rounded weights.  P is rounded to bf16 for the
+// MMA; O is divided by the sum of those rounded values (so O is a weighted
+// mean with exactly the weights used) and the LSE uses the unrounded sum.
+// The row max is taken over the first two 32-column loads of S while the last
+// two are still in flight.
 //
 // Mask variants ("flash-attention" skill page, section 3.3), compiled into a
 // second instantiation (GENERAL = true) so the plain causal / full kernel
@@ -98,7 +103,7 @@ static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= NUM_THREADS * kRegsLaun
               "register split exceeds the launch allocation");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
-constexpr int MAX_LEVELS = 1024;  // max_seqlen <= 1024 * 256
+constexpr int MAX_LEVELS = 4096;  // max_seqlen <= 4096 * 256
 constexpr int MAX_ITEMS_PER_CTA = 192;
 constexpr int SMEM_LIMIT = 232448;  // dynamic shared memory per CTA on sm_100
 
@@ -125,8 +130,8 @@ struct Cfg {
   static constexpr int PV_KSTEPS = BN / KSTEP;        // MMAs per P V tile
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = NQT * TILE_BYTES;
-  // O leaves through a bf16 staging panel per query tile (64 columns x 128
-  // rows, 128-byte swizzle), one TMA store per panel
+  // O leaves through a 4 KB bf16 staging region per softmax warp (32 rows x
+  // 64 columns), 16 KB per query tile
   static constexpr int O_PANEL_BYTES = BM * 128;
   static constexpr int O_PANELS = D / 64;
   static constexpr int O_STAGE_OFF = KV_OFF + STAGES * TILE_BYTES;
@@ -210,9 +215,7 @@ struct Shared {
   uint64_t kv_full[8], kv_empty[8];
   uint64_t s_full[NQT], o_full[NQT];
   uint64_t p_full[NQT][P_CHUNKS];  // one chunk of P written to TMEM
-  // O staging panel of each query tile: written by the tile's 128 threads
-  // (stage_full), read out by the TMA store (stage_free)
-  uint64_t stage_full[NQT], stage_free[NQT];
+  uint64_t stall;                  // never arrived at (timeout test hook)
   uint32_t tmem_base;
   int abort;
   int num_items;                     // items this CTA processes
@@ -221,15 +224,17 @@ struct Shared {
 };
 
 // Work-list construction scratch; only live before the main loop, so it
-// shares its shared memory with the O staging panels.
+// shares its shared memory with the K/V ring (which the first TMA load
+// overwrites after the prologue).
 struct PlanScratch {
-  int level_count[MAX_LEVELS];       // sequences with more than l 256-row blocks
+  int hist[MAX_LEVELS + 1];          // sequences with exactly n 256-row blocks
   int level_offset[MAX_LEVELS + 1];  // first item index of level (descending order)
 };
 
 template <int D, bool FP8 = false>
 constexpr int smem_bytes() {
-  static_assert(sizeof(PlanScratch) <= NQT * Cfg<D, FP8>::O_PANEL_BYTES, "plan scratch overflows");
+  static_assert(sizeof(PlanScratch) <= Cfg<D, FP8>::STAGES * Cfg<D, FP8>::TILE_BYTES,
+                "plan scratch overflows the K/V ring");
   return Cfg<D, FP8>::SMEM_TILES + (int)sizeof(Shared) + 1024;
 }
 static_assert(smem_bytes<128>() <= SMEM_LIMIT && smem_bytes<64>() <= SMEM_LIMIT &&
@@ -276,12 +281,6 @@ __device__ __forceinline__ void item_kv_range(const Params& p, int q0, int len, 
   }
 }
 
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
 // Length of sequence b as the kernel uses it: an inconsistent cu_seqlens
 // entry reports a bounds error and makes the sequence empty.
 __device__ __forceinline__ void seq_range(const Params& p, int b, int& start, int& len) {
@@ -294,6 +293,14 @@ __device__ __forceinline__ void seq_range(const Params& p, int b, int& start, in
   }
   start = s;
   len = e - s;
+}
+
+// Sum of the four lanes of two packed fp32 pairs.
+__device__ __forceinline__ float sum4(uint64_t a, uint64_t b) {
+  float a0, a1, b0, b1;
+  f2_unpack(a, a0, a1);
+  f2_unpack(b, b0, b1);
+  return (a0 + a1) + (b0 + b1);
 }
 
 __device__ __forceinline__ int blocks_of(int len) { return (len + ROWS_PER_ITEM - 1) / ROWS_PER_ITEM; }
@@ -332,10 +339,12 @@ __device__ void decode_item(const Params& p, const PlanScratch& sh, int w, int& 
 template <int D, bool GENERAL, bool FP8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const __grid_constant__ CUtensorMap tmV,
                    const Params p) {
   using C = Cfg<D, FP8>;
   static_assert(!(GENERAL && FP8), "mask variants are not built for e4m3");
+  // one exp2 pair in POLY_EVERY on the FMA pipe, the rest on MUFU (0: all MUFU)
+  constexpr int POLY_EVERY = 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -343,7 +352,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* kv_smem = smem + C::KV_OFF;
   uint8_t* o_stage = smem + C::O_STAGE_OFF;
   Shared& sh = *reinterpret_cast<Shared*>(smem + C::SMEM_TILES);
-  PlanScratch& ps = *reinterpret_cast<PlanScratch*>(o_stage);
+  PlanScratch& ps = *reinterpret_cast<PlanScratch*>(kv_smem);
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -356,6 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&sh.q_empty[t], 1);
     }
     mbar_init(&sh.mma_done, 1);
+    mbar_init(&sh.stall, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&sh.kv_full[s], 1);
       mbar_init(&sh.kv_empty[s], 1);
@@ -364,8 +374,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&sh.s_full[t], 1);
       for (int c = 0; c < P_CHUNKS; ++c) mbar_init(&sh.p_full[t][c], BM);
       mbar_init(&sh.o_full[t], 1);
-      mbar_init(&sh.stage_full[t], BM);
-      mbar_init(&sh.stage_free[t], 1);
     }
     sh.abort = 0;
     fence_mbar_init();
@@ -374,13 +382,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  for (int l = tid; l < p.num_levels; l += NUM_THREADS) ps.level_count[l] = 0;
+  for (int l = tid; l <= p.num_levels; l += NUM_THREADS) ps.hist[l] = 0;
   __syncthreads();
   for (int b = tid; b < p.B; b += NUM_THREADS) {
     int st, len;
@@ -393,14 +400,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       nb = p.num_levels;
     }
     // level l holds sequence b for every l < nb
-    for (int l = 0; l < nb; ++l) atomicAdd(&ps.level_count[l], 1);
+    atomicAdd(&ps.hist[nb], 1);
   }
   __syncthreads();
   if (tid == 0) {
-    int acc = 0;
+    // level l holds the sequences with more than l blocks: sum of hist[n], n > l
+    int acc = 0, cnt = 0;
     for (int k = 0; k < p.num_levels; ++k) {
+      cnt += ps.hist[p.num_levels - k];
       ps.level_offset[k] = acc;
-      acc += ps.level_count[p.num_levels - 1 - k] * p.Hq;
+      acc += cnt * p.Hq;
     }
     ps.level_offset[p.num_levels] = acc;
     sh.total_items = acc;
@@ -426,6 +435,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     decode_item(p, ps, w, b, level, h);
     sh.items[i] = make_int2(b, (level << 16) | h);
   }
+  // the plan scratch was written through the generic proxy; the ring's TMA
+  // loads (async proxy) overwrite it after the barrier below
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -696,7 +708,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t s_col = lane_base + t * 128;
     const uint32_t o_col = lane_base + 256 + t * 128;
     uint32_t s_phase = 0, o_phase = 0;
-    uint32_t n_stage = 0;  // O panels staged by this group so far
+    // timeout test hook: this group's first S wait is on a barrier that
+    // nothing arrives at
+    bool stall = t == 0 && blockIdx.x == 0 &&
+                 *reinterpret_cast<volatile int*>(&g_stall_test) == kStallPrefill;
     const float sl = p.scale_log2;
     const uint64_t sl2 = f2_pack(sl, sl);
     bool ok = true;
@@ -715,108 +730,124 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           (GENERAL && p.alibi) ? __ldg(p.alibi + (size_t)b * p.alibi_stride + h) * 1.4426950408889634f
                                : 0.f;
       float m_ref = -INFINITY;
-      // row sums, each as two interleaved fp32 pairs: le = exact sum of
-      // exp (for the LSE), lr = sum of the bf16 values the PV MMA consumes
-      // (normalises O consistently with its own weights)
+      // Row sums as interleaved fp32 pairs.  le: the unrounded weights (gives
+      // the LSE).  O is normalised by the sum of the weights the P V MMA
+      // consumed on every tile that needs masking (where rows with few
+      // visible keys live) and by the unrounded weights elsewhere: bf16 keeps
+      // that as le + corr, corr = sum over masked tiles of (rounded -
+      // unrounded), from the per-tile rounded sums lr; e4m3 (whose rounding
+      // is coarser) sums its decoded weights on every tile into lr.
       uint64_t le_a = 0, le_b = 0;
       float lr_a0 = 0.f, lr_a1 = 0.f, lr_b0 = 0.f, lr_b1 = 0.f;
+      float corr = 0.f;
       for (int j = jlo; j < jhi; ++j) {
-        if (!mbar_wait(&sh.s_full[t], s_phase, abort)) { ok = false; break; }
+        if (!mbar_wait(stall ? &sh.stall : &sh.s_full[t], s_phase, abort)) { ok = false; break; }
+        stall = false;
         s_phase ^= 1;
         tc_fence_after();
         uint32_t s[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, s[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_wait(s[c]);
         const int kv0 = j * BN;
+        // masking of chunk c (32 columns): keys outside [0, len) or outside
+        // the row's band (GENERAL), keys past the sequence end or after the
+        // query (plain)
+        bool need_mask;
+        int lim_lo = -1, lim_hi = BN;  // visible columns [lim_lo, lim_hi)
         if constexpr (GENERAL) {
-          // logits in log2 units: optional cap, then the ALiBi distance penalty
-          if (p.cap_out > 0.f) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                // tanh(y) = 1 - 2 / (1 + 2^(2 y log2 e)); saturates to +-1
-                const float big = ex2(__uint_as_float(s[c][e]) * p.cap_in);
-                const float th = fmaf(-2.f, rcp_approx(1.f + big), 1.f);
-                s[c][e] = __float_as_uint(th * p.cap_out);
-              }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-              for (int e = 0; e < 32; ++e) s[c][e] = __float_as_uint(__uint_as_float(s[c][e]) * sl);
-          }
-          if (slope2 != 0.f) {
-            const float d0 = (float)(kv0 - qpos);  // key - query for column 0
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                s[c][e] = __float_as_uint(
-                    fmaf(-slope2, fabsf(d0 + (float)(c * 32 + e)), __uint_as_float(s[c][e])));
-          }
-          // masking: keys outside [0, len) or outside the row's band
-          if (kv0 + BN > len || (p.wr >= 0 && kv0 + BN - 1 > rs + p.wr) ||
-              (p.wl >= 0 && kv0 < rs + BM - 1 - p.wl)) {
-            const int lim_lo = p.wl >= 0 ? qpos - p.wl - kv0 : -1;  // columns [lim_lo, lim_hi)
-            const int lim_hi = min(len, p.wr >= 0 ? qpos + p.wr + 1 : len) - kv0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                s[c][e] = (c * 32 + e < lim_lo || c * 32 + e >= lim_hi)
-                              ? __float_as_uint(-INFINITY) : s[c][e];
-          }
+          need_mask = kv0 + BN > len || (p.wr >= 0 && kv0 + BN - 1 > rs + p.wr) ||
+                      (p.wl >= 0 && kv0 < rs + BM - 1 - p.wl);
+          lim_lo = p.wl >= 0 ? qpos - p.wl - kv0 : -1;
+          lim_hi = min(len, p.wr >= 0 ? qpos + p.wr + 1 : len) - kv0;
         } else {
-          // masking: keys past the sequence end, and (causal) keys after the query
-          if (kv0 + BN > len || (p.causal && kv0 + BN - 1 > rs)) {
-            const int lim = min(len, p.causal ? qpos + 1 : len) - kv0;  // keys [0, lim) visible
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
+          need_mask = kv0 + BN > len || (p.causal && kv0 + BN - 1 > rs);
+          lim_hi = min(len, p.causal ? qpos + 1 : len) - kv0;
+        }
+        // GENERAL: logits in log2 units (optional cap, then the ALiBi
+        // penalty), then the band mask; plain: the mask only
+        auto prepare = [&](uint32_t (&x)[32], int c) {
+          if constexpr (GENERAL) {
+            if (p.cap_out > 0.f) {
 #pragma unroll
               for (int e = 0; e < 32; ++e)
-                s[c][e] = (c * 32 + e >= lim) ? __float_as_uint(-INFINITY) : s[c][e];
+                x[e] = __float_as_uint(softcap_log2(__uint_as_float(x[e]), p.cap_in, p.cap_out));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) x[e] = __float_as_uint(__uint_as_float(x[e]) * sl);
+            }
+            if (slope2 != 0.f) {
+              const float d0 = (float)(kv0 + c * 32 - qpos);  // key - query for column 0 of the chunk
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                x[e] = __float_as_uint(
+                    fmaf(-slope2, fabsf(d0 + (float)e), __uint_as_float(x[e])));
+            }
           }
-        }
-        // row max: eight independent chains of three-input maxima (short
-        // chains: the max is on the tile's critical path)
+          if (need_mask) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              x[e] = (c * 32 + e < lim_lo || c * 32 + e >= lim_hi) ? __float_as_uint(-INFINITY)
+                                                                  : x[e];
+          }
+        };
+        // row max: four independent chains of three-input maxima per pair of
+        // chunks; the max of chunks 0-1 runs while chunks 2-3 load
         float mx[8];
+        auto chunk_max = [&](const uint32_t (&a)[32], const uint32_t (&b)[32], float* m) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mx[k] = fmaxf(__uint_as_float(s[k >> 1][(k & 1) * 16]), __uint_as_float(s[k >> 1][(k & 1) * 16 + 1]));
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t* src = (k < 2) ? a : b;
+            const int o = (k & 1) * 16;
+            m[k] = fmaxf(__uint_as_float(src[o]), __uint_as_float(src[o + 1]));
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-#pragma unroll
-          for (int e = 2; e < 16; e += 2)
-            mx[k] = fmax3(mx[k], __uint_as_float(s[k >> 1][(k & 1) * 16 + e]),
-                          __uint_as_float(s[k >> 1][(k & 1) * 16 + e + 1]));
+            for (int e = 2; e < 16; e += 2)
+              m[k] = fmax3(m[k], __uint_as_float(src[o + e]), __uint_as_float(src[o + e + 1]));
+          }
+        };
+        tmem_ld32(s_col, s[0]);
+        tmem_ld32(s_col + 32, s[1]);
+        tmem_ld_wait(s[0]);
+        tmem_ld_tie(s[1]);
+        tmem_ld32(s_col + 64, s[2]);
+        tmem_ld32(s_col + 96, s[3]);
+        prepare(s[0], 0);
+        prepare(s[1], 1);
+        chunk_max(s[0], s[1], mx);
+        tmem_ld_wait(s[2]);
+        tmem_ld_tie(s[3]);
+        prepare(s[2], 2);
+        prepare(s[3], 3);
+        chunk_max(s[2], s[3], mx + 4);
         const float mx_s = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
                                  fmaxf(mx[6], mx[7])) * (GENERAL ? 1.f : sl);
+        // Lazy rescale, decided per row: the reference max moves only when the
+        // tile max exceeds it by more than the threshold.  The exponentials
+        // start at once with this row's reference; O is rescaled in tensor
+        // memory (a warp-wide pass, if any row of the warp moved) just before
+        // the first chunk of P is released.
         float alpha = 1.f;
-        bool rescale = false;
+        bool moved = false;
         if (j == jlo) {
           // GENERAL keeps -inf for a row that sees nothing in this tile
           m_ref = (!GENERAL && mx_s == -INFINITY) ? 0.f : mx_s;
-        } else if (__any_sync(0xffffffffu, mx_s > m_ref + kRescaleThreshold)) {
+        } else if (mx_s > m_ref + kRescaleThreshold) {
           const float m_new = fmaxf(m_ref, mx_s);
           // (m_ref == m_new also covers -inf == -inf, where the difference is NaN)
           alpha = (GENERAL && m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
+          m_ref = m_new;
+          moved = true;
           const uint64_t a2 = f2_pack(alpha, alpha);
           le_a = f2_mul(le_a, a2);
           le_b = f2_mul(le_b, a2);
+          corr *= alpha;
           lr_a0 *= alpha;
           lr_a1 *= alpha;
           lr_b0 *= alpha;
           lr_b1 *= alpha;
-          m_ref = m_new;
-          rescale = true;
         }
-        if (rescale) {
-          // O *= alpha before any chunk of P is released: every P V of step j-1
-          // has completed (they precede S_t(j) in issue order).  16 columns at
-          // a time, since all of S is still held in registers here.
+        const bool rescale = j != jlo && __any_sync(0xffffffffu, moved);
+        auto rescale_o = [&]() {
+          // O *= alpha: every P V of step j-1 has completed (they precede
+          // S_t(j) in issue order) and none of step j has started.  16
+          // columns at a time, since S is still held in registers here.
           const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
           for (int c = 0; c < D / 16; ++c) {
@@ -832,13 +863,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             tmem_st16(o_col + c * 16, o);
           }
-        }
-        // P = 2^(s*scale*log2e - m): three of every four pairs on MUFU, one on
-        // the FMA pipe; packed bf16 pairs overwrite s[c][0..15] in order
+        };
+        // P = 2^(s*scale*log2e - m); packed bf16 (or e4m3) pairs overwrite
+        // s[c][0..] in order
         const float m_use = (GENERAL && m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t neg2 = f2_pack(-m_use, -m_use);
         // GENERAL: s already holds scaled logits, so the FMA multiplies by 1
         const uint64_t mul2 = GENERAL ? f2_pack(1.f, 1.f) : sl2;
+        // Tiles whose normaliser takes the rounded weights (see the row sums
+        // above): every e4m3 tile, every tile of the mask variants (whose
+        // rows often hold few effective keys), the masked tiles of the plain
+        // kernel.  For bf16 the rounded weights of a quarter are summed from
+        // its packed words after its exponentials, so full tiles run the same
+        // exponential code without that work.
+        const bool round = FP8 || GENERAL || need_mask;
+        float le_tile0 = 0.f;
+        if (!FP8 && round) {
+          le_tile0 = sum4(le_a, le_b);
+          lr_a0 = lr_a1 = lr_b0 = lr_b1 = 0.f;
+        }
         uint32_t e4_lo = 0;  // e4m3: the even pair of a word, waiting for the odd one
         // four 32-key quarters; a chunk is 4 / P_CHUNKS consecutive quarters
         constexpr int QPC = 4 / P_CHUNKS;
@@ -849,7 +892,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t x =
                 f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), mul2, neg2);
             uint64_t pr;
-            if (((e >> 1) & 3) == 3) {
+            if (POLY_EVERY > 0 && ((e >> 1) % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
               pr = exp2_fma_pair(x);
             } else {
               float x0, x1;
@@ -858,35 +901,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             float p0, p1;
             f2_unpack(pr, p0, p1);
+            if ((e >> 1) & 1) le_b = f2_add(le_b, pr); else le_a = f2_add(le_a, pr);
             if constexpr (FP8) {
               // four e4m3 per word: pairs 2w and 2w+1 of the chunk form word w
               const uint32_t pq = pack_e4m3x2(p0, p1);
               if ((e >> 1) & 1) {
-                le_b = f2_add(le_b, pr);
                 add_e4m3x2_f32(pq, lr_b0, lr_b1);
                 s[c][e >> 2] = e4_lo | (pq << 16);
               } else {
-                le_a = f2_add(le_a, pr);
                 add_e4m3x2_f32(pq, lr_a0, lr_a1);
                 e4_lo = pq;
               }
             } else {
-              const uint32_t pp = pack_bf16x2(p0, p1);
-              if ((e >> 1) & 1) {
-                le_b = f2_add(le_b, pr);
-                lr_b0 = add_bf16lo_f32(pp, lr_b0);
-                lr_b1 = add_bf16hi_f32(pp, lr_b1);
-              } else {
-                le_a = f2_add(le_a, pr);
-                lr_a0 = add_bf16lo_f32(pp, lr_a0);
-                lr_a1 = add_bf16hi_f32(pp, lr_a1);
-              }
-              s[c][e >> 1] = pp;
+              s[c][e >> 1] = pack_bf16x2(p0, p1);
+            }
+          }
+          if (!FP8 && round) {
+#pragma unroll
+            for (int w = 0; w < 16; w += 2) {
+              lr_a0 = add_bf16lo_f32(s[c][w], lr_a0);
+              lr_a1 = add_bf16hi_f32(s[c][w], lr_a1);
+              lr_b0 = add_bf16lo_f32(s[c][w + 1], lr_b0);
+              lr_b1 = add_bf16hi_f32(s[c][w + 1], lr_b1);
             }
           }
           // the chunk that ended with quarter c-1 has had this quarter's math
-          // to land: release it, then store quarter c
+          // to land: release it (after the O rescale, before the first
+          // release), then store quarter c
           if (c > 0 && c % QPC == 0) {
+            if (c == QPC && rescale) rescale_o();
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&sh.p_full[t][c / QPC - 1]);
@@ -896,6 +939,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           else
             tmem_st16(s_col + c * 16, s[c]);
         }
+        if (QPC == 4 && rescale) rescale_o();
+        // bf16: the normaliser takes this tile's rounded weights:
+        // corr += sum(rounded) - sum(unrounded) over the tile
+        if (!FP8 && round)
+          corr += ((lr_a0 + lr_a1) + (lr_b0 + lr_b1)) - (sum4(le_a, le_b) - le_tile0);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sh.p_full[t][P_CHUNKS - 1]);
@@ -909,84 +957,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       f2_unpack(le_a, la0, la1);
       f2_unpack(le_b, lb0, lb1);
       const float l_exact = (la0 + la1) + (lb0 + lb1);
-      const float l_round = (lr_a0 + lr_a1) + (lr_b0 + lr_b1);
+      const float l_norm = FP8 ? (lr_a0 + lr_a1) + (lr_b0 + lr_b1) : l_exact + corr;
       const bool valid = qpos < len;
-      const float inv_l = p.o_scale / l_round;
+      const float inv_l = p.o_scale / l_norm;
       const size_t grow = (size_t)(start + qpos);
-      if (rs + BM <= len) {
-        // full tile: each 64-column panel is normalised into the staging
-        // panel (row = this thread's row, 16-byte chunks swizzled by row & 7)
-        // and written by one TMA store, so no thread waits on global stores
-        uint8_t* stage = o_stage + t * C::O_PANEL_BYTES;
-        uint8_t* srow = stage + row * 128;
+      // Each warp writes its own 32 rows, one 64-column panel at a time:
+      // every thread puts its row into the warp's 4 KB staging region
+      // (16-byte chunks XOR-swizzled by row, so neither the writes nor the
+      // reads conflict on banks), then the warp reads it back four rows per
+      // instruction, eight lanes per row, for 128-byte global stores.  Rows
+      // past the sequence end are not stored; every lane takes part in the
+      // warp-wide TMEM loads.  Only __syncwarp orders the staging.
+      uint8_t* wst = o_stage + (t * 4 + quarter) * 4096;
+      const int rbase = rs + quarter * 32;  // local row of the warp's lane 0
 #pragma unroll
-        for (int pn = 0; pn < C::O_PANELS; ++pn) {
-          uint32_t o[2][32];
-          tmem_ld32(o_col + pn * 64, o[0]);
-          tmem_ld32(o_col + pn * 64 + 32, o[1]);
-          tmem_ld_wait(o[0]);
-          tmem_ld_wait(o[1]);
-          // the previous store from this panel must have read it out
-          if (n_stage > 0 && !mbar_wait(&sh.stage_free[t], (n_stage - 1) & 1, abort)) {
-            ok = false;
-            break;
-          }
+      for (int pn = 0; pn < C::O_PANELS; ++pn) {
+        uint32_t o[2][32];
+        tmem_ld32(o_col + pn * 64, o[0]);
+        tmem_ld32(o_col + pn * 64 + 32, o[1]);
+        tmem_ld_wait(o[0]);
+        tmem_ld_tie(o[1]);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t* src = o[c >> 2] + (c & 3) * 8;
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(src[0]) * inv_l, __uint_as_float(src[1]) * inv_l);
-            v.y = pack_bf16x2(__uint_as_float(src[2]) * inv_l, __uint_as_float(src[3]) * inv_l);
-            v.z = pack_bf16x2(__uint_as_float(src[4]) * inv_l, __uint_as_float(src[5]) * inv_l);
-            v.w = pack_bf16x2(__uint_as_float(src[6]) * inv_l, __uint_as_float(src[7]) * inv_l);
-            *reinterpret_cast<uint4*>(srow + ((c ^ (row & 7)) << 4)) = v;
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&sh.stage_full[t]);
-          bool stored = true;
-          if (row == 0) {
-            stored = mbar_wait(&sh.stage_full[t], n_stage & 1, abort);
-            if (stored) {
-              tma_store_2d(&tmO, stage, h * D + pn * 64, start + rs);
-              bulk_commit_group();
-              bulk_wait_read_all();
-              mbar_arrive(&sh.stage_free[t]);
-            }
-          }
-          ++n_stage;
-          if (!__all_sync(0xffffffffu, stored)) {
-            ok = false;
-            break;
-          }
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t* src = o[c >> 2] + (c & 3) * 8;
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(src[0]) * inv_l, __uint_as_float(src[1]) * inv_l);
+          v.y = pack_bf16x2(__uint_as_float(src[2]) * inv_l, __uint_as_float(src[3]) * inv_l);
+          v.z = pack_bf16x2(__uint_as_float(src[4]) * inv_l, __uint_as_float(src[5]) * inv_l);
+          v.w = pack_bf16x2(__uint_as_float(src[6]) * inv_l, __uint_as_float(src[7]) * inv_l);
+          *reinterpret_cast<uint4*>(wst + lane * 128 + ((c ^ (lane & 7)) << 4)) = v;
         }
-        if (!ok) break;
-      } else {
-        // the tile runs past the sequence end: rows are stored one by one
-        // (every lane takes part in the warp-wide TMEM loads)
-        uint4* dst = reinterpret_cast<uint4*>(p.o + (grow * p.Hq + h) * D);
+        __syncwarp();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_col + c * 32, o);
-          tmem_ld_wait(o);
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
-                               __uint_as_float(o[2 * e + 1]) * inv_l);
-          if (valid) {
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              dst[c * 4 + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
-          }
+        for (int i = 0; i < 8; ++i) {
+          const int r = i * 4 + (lane >> 3);  // row of the warp
+          const int c = lane & 7;             // 16-byte chunk of its 128 bytes
+          const uint4 v = *reinterpret_cast<const uint4*>(wst + r * 128 + ((c ^ (r & 7)) << 4));
+          if (rbase + r < len)
+            *reinterpret_cast<uint4*>(p.o + ((size_t)(start + rbase + r) * p.Hq + h) * D +
+                                      pn * 64 + c * 8) = v;
         }
+        __syncwarp();
       }
       if (valid && p.lse)
         p.lse[(size_t)h * p.T + grow] = (m_ref + __log2f(l_exact)) * 0.69314718055994531f;
       tc_fence_before();
     }
-    // the staged O stores must be complete before the CTA exits
-    if (row == 0) bulk_wait_all();
   }
 
   // ---------------- teardown ----------------

@@ -48,6 +48,10 @@ extern "C" {
 
 typedef struct CUstream_st *fa_stream_t; /* identical to cudaStream_t */
 
+/* Largest batch whose decode plan (the prefix sums of the per-request range
+ * counts) each CTA of the decode's split kernel builds itself. */
+#define FA_DECODE_PLAN_MAX_B 2048
+
 typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARG = 1,    /* null pointer, bad shape, misalignment       */
@@ -72,11 +76,14 @@ typedef enum {
  *               zero: it sees all L_b keys of its own sequence
  *   scale       multiplier of Q K^T (<= 0: 1/sqrt(d))
  *   total_tokens  T (host copy of cu_seqlens[B]; sizes q/k/v/o)
- *   max_seqlen    an upper bound on every L_b (host): sizes the device work
- *                 list of 256-row blocks.  At most 262144
- *                 (FA_ERR_UNSUPPORTED above).  For a sequence longer than
- *                 ceil(max_seqlen / 256) * 256 rows, the rows past that are
- *                 not computed (their O and LSE are left as they were) and
+ *   max_seqlen    optional hint (the pages' max_seqlen_q/k): an upper bound
+ *                 on every L_b, known on the host, that sizes the device work
+ *                 list of 256-row blocks.  <= 0 = not given: the library uses
+ *                 min(T, 1048576), which always holds when T <= 1048576.  At
+ *                 most 1048576 (FA_ERR_UNSUPPORTED above).  A hint smaller
+ *                 than the longest sequence is an error the device reports:
+ *                 the rows past ceil(max_seqlen / 256) * 256 are not computed
+ *                 (their O and LSE are left as they were) and
  *                 FA_ERR_DEVICE_BOUNDS is set.
  * Query head h reads kv head h / (Hq / Hkv); Hq <= 65535.  A sequence with
  * L_b = 0 is skipped.  The grid is one CTA per SM, widened when a CTA would
@@ -160,8 +167,16 @@ fa_status fa_prefill_fp8(const void *q, const void *k, const void *v, void *o, f
  *                fa_decode_workspace_size(B, Hq, d, resolved num_splits)
  *                bytes, 256-byte aligned; NULL = the library allocates it
  *                stream-ordered (cudaMallocAsync/cudaFreeAsync on `stream`)
- * A request with seq_lens[b] = 0 yields O = 0 and LSE = -inf.  Requires
- * Hq / Hkv <= 8.
+ * A request with seq_lens[b] = 0 yields O = 0 and LSE = -inf; num_pages may
+ * be 0 when every context is empty (the pool is then never read).  Any
+ * group size Hq / Hkv and any page_size >= 1 are taken: a page size that is
+ * a multiple of 16 is gathered with TMA boxes of 16 tokens, any other token
+ * by token with 16-byte copies.  Each K/V byte is read from device memory
+ * once per kv head for groups of up to 64 query heads (once per 64 query
+ * heads above that).  Kernels launched: the split kernel, then, when a
+ * request can have more than one range, the LSE combine (a programmatic
+ * dependent launch of the split kernel), and before them, for
+ * B > FA_DECODE_PLAN_MAX_B with more than one range, a one-CTA plan kernel.
  */
 fa_status fa_decode_paged(const void *q, const void *k_pages, const void *v_pages,
                           const int32_t *block_table, const int32_t *seq_lens, int page_size,
@@ -269,6 +284,45 @@ fa_status fa_decode_paged_f32(const float *q, const float *k_pages, const float 
                               int page_size, float *o, fa_stream_t stream, int B, int Hq,
                               int Hkv, int d, int max_blocks_per_seq, int num_pages,
                               float scale, float *lse);
+
+/*
+ * Self-test hook (used by the tests, not by the attention path): evaluates
+ * on the GPU, element by element, a scalar function the prefill kernel
+ * computes its softmax weights with, so it can be compared with an exact
+ * reference over its whole input range.
+ *
+ *   op  FA_MATH_EXP2_FMA:     2^x on the FMA pipe (range reduction plus the
+ *                             cubic of exp2_poly.cuh); x < -126 gives 0
+ *       FA_MATH_EXP2_MUFU:    2^x by ex2.approx.ftz (the MUFU unit)
+ *       FA_MATH_SOFTCAP_LOG2: a * b-scaled tanh: b * tanh(x * a / (2 log2 e)),
+ *                             i.e. the softcapped logit in log2 units with
+ *                             a = 2 log2(e) scale / cap and b = cap log2(e)
+ *   x, y  fp32 [n], device; y = f(x) (written)
+ * Returns FA_ERR_INVALID_ARG for an unknown op or n < 0.
+ */
+enum { FA_MATH_EXP2_FMA = 0, FA_MATH_EXP2_MUFU = 1, FA_MATH_SOFTCAP_LOG2 = 2 };
+fa_status fa_selftest_math(int op, const float *x, float *y, int n, float a, float b,
+                           fa_stream_t stream);
+
+/*
+ * Self-test hook (used by the tests of the timeout path, not by the
+ * attention path): sets, for the current device, which kernel makes one
+ * warp of its first CTA wait on a barrier that nothing arrives at, and the
+ * time limit of the kernels' abortable waits.
+ *
+ *   which          0 = none (normal operation), FA_STALL_PREFILL = the first
+ *                  softmax warpgroup of the prefill kernels (its first wait
+ *                  for S), FA_STALL_DECODE = the first consumer warp of the
+ *                  decode split kernel (its first wait for a stage)
+ *   wait_limit_ns  limit of the abortable waits; 0 = the default, 2 s
+ * When the limit runs out the kernel records FA_ERR_DEVICE_TIMEOUT, its
+ * other roles stop, it waits (up to 2 s, whatever wait_limit_ns says) for
+ * its own copies and tensor-core work in flight, frees its tensor memory and
+ * returns; the outputs of that call are unspecified.  Synchronous (writes
+ * two device variables).  Call with (0, 0) to restore normal operation.
+ */
+enum { FA_STALL_PREFILL = 1, FA_STALL_DECODE = 2 };
+fa_status fa_selftest_inject_stall(int which, unsigned long long wait_limit_ns);
 
 /* Reads and clears the sticky device error word of the current device
  * (synchronises `stream` first).  *code receives FA_OK or the first
