@@ -3,11 +3,13 @@
 Tolerances: bf16 outputs within max-abs 1e-2 and mean-abs 1e-3 of the fp64
 oracle, LSE within 1e-3; the fp32 debug path within 1e-5.
 
-The mean bound on bf16 outputs is applied on top of the mean error that
+check_bf16_plain applies exactly those bounds; the five named workloads
+use it.  check_bf16 applies the mean bound on top of the mean error that
 rounding the exact (fp64) result once to bf16 already has, mean|bf16(ref) -
-ref|: no bf16 output can do better than that.  For rows that average many
-keys |O| is small and this floor is ~1e-4; for rows of one or two keys |O| is
-O(1) and the floor alone is ~1e-3.
+ref|, since no bf16 output can do better than that: for rows that average
+many keys |O| is small and this floor is ~1e-4, but for rows of one or two
+keys |O| is O(1) and the floor alone is ~1e-3, so the stress shapes with
+such rows (single sequences of 1..3 tokens, tiny windows) use it.
 """
 import numpy as np
 import torch
@@ -31,6 +33,11 @@ def bf16_rounding_floor(ref):
     r = ref[fin]
     rb = torch.from_numpy(r).to(torch.bfloat16).double().numpy()
     return float(np.abs(rb - r).mean())
+
+
+def check_bf16_plain(got, ref, what="O"):
+    """The bf16 output bounds exactly as stated: max-abs 1e-2, mean-abs 1e-3."""
+    return check_close(got, ref, BF16_MAX_ABS, BF16_MEAN_ABS, what)
 
 
 def check_bf16(got, ref, what="O"):

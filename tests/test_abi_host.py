@@ -69,7 +69,7 @@ def test_prefill_argument_checks(lib):
     assert _prefill(lib, q=ctypes.c_void_p(0x1008)) == api.FA_ERR_INVALID_ARG  # misaligned
     assert _prefill(lib, d=96) == api.FA_ERR_UNSUPPORTED
     assert _prefill(lib, d=256) == api.FA_ERR_UNSUPPORTED
-    assert _prefill(lib, maxlen=1024 * 256 + 1) == api.FA_ERR_UNSUPPORTED
+    assert _prefill(lib, maxlen=4096 * 256 + 1) == api.FA_ERR_UNSUPPORTED
     assert _prefill(lib, Hq=65536, Hkv=1) == api.FA_ERR_UNSUPPORTED   # head index is 16-bit
     # empty problems are a no-op (no launch)
     assert _prefill(lib, B=0) == api.FA_OK
@@ -116,7 +116,7 @@ def test_prefill_fp8_argument_checks(lib):
         assert _prefill_fp8(lib, vd=bad) == api.FA_ERR_INVALID_ARG
     assert _prefill_fp8(lib, d=64) == api.FA_ERR_UNSUPPORTED           # e4m3 path is d = 128
     assert _prefill_fp8(lib, Hq=65536, Hkv=1) == api.FA_ERR_UNSUPPORTED
-    assert _prefill_fp8(lib, maxlen=1024 * 256 + 1) == api.FA_ERR_UNSUPPORTED
+    assert _prefill_fp8(lib, maxlen=4096 * 256 + 1) == api.FA_ERR_UNSUPPORTED
     assert _prefill_fp8(lib, B=0) == api.FA_OK
     assert _prefill_fp8(lib, T=0) == api.FA_OK
 
@@ -137,8 +137,6 @@ def test_decode_argument_checks(lib):
     assert _decode(lib, Hq=12, Hkv=8) == api.FA_ERR_INVALID_ARG
     assert _decode(lib, ws=ctypes.c_void_p(0x1010)) == api.FA_ERR_INVALID_ARG  # not 256-aligned
     assert _decode(lib, d=80) == api.FA_ERR_UNSUPPORTED
-    assert _decode(lib, Hq=32, Hkv=2) == api.FA_ERR_UNSUPPORTED          # group 16 > 8
-    assert _decode(lib, ps=8) == api.FA_ERR_UNSUPPORTED                  # not a multiple of 16
     # explicit workspace that is too small
     need = lib.fa_decode_workspace_size(2, 32, 128, 4)
     assert _decode(lib, S=4, ws=ctypes.c_void_p(0x10000), wsb=need - 1) == api.FA_ERR_INVALID_ARG
@@ -164,7 +162,6 @@ def test_decode_append_argument_checks(lib):
     assert _append(lib, cos=FAKE, sin=FAKE, maxpos=10, rd=130) == api.FA_ERR_INVALID_ARG  # > d
     assert _append(lib, cos=FAKE, sin=FAKE, maxpos=0, rd=64) == api.FA_ERR_INVALID_ARG
     assert _append(lib, d=96) == api.FA_ERR_UNSUPPORTED
-    assert _append(lib, ps=8) == api.FA_ERR_UNSUPPORTED
     need = lib.fa_decode_append_workspace_size(2, 32, 128, 4)
     assert need == (lib.fa_decode_workspace_size(2, 32, 128, 4) + 2 * 32 * 128 * 2 + 256)
     assert _append(lib, S=4, ws=ctypes.c_void_p(0x10000), wsb=need - 1) == api.FA_ERR_INVALID_ARG
@@ -205,3 +202,40 @@ def test_python_binding_rejects_host_tensors():
     cu = torch.tensor([0, 4], dtype=torch.int32)
     with pytest.raises(ValueError):
         api.fa_prefill(q, q[:, :1], q[:, :1], q, None, cu, True)
+
+
+@pytest.mark.parametrize("which", ["fa_decode_paged", "fa_decode_paged_noalloc",
+                                   "fa_decode_paged_append"])
+def test_decode_wrappers_check_the_output_shapes(which):
+    """The decode kernels write B*Hq*d elements of o and B*Hq of lse, so each
+    decode wrapper refuses an o or lse of another shape before any call
+    (a smaller buffer would be written past its end)."""
+    import torch
+    B, Hq, Hkv, d, ps = 3, 8, 2, 64, 16
+    bf = torch.bfloat16
+    q = torch.zeros(B, Hq, d, dtype=bf)
+    kp = torch.zeros(4, ps, Hkv, d, dtype=bf)
+    bt = torch.zeros(B, 2, dtype=torch.int32)
+    sl = torch.zeros(B, dtype=torch.int32)
+    kn = torch.zeros(B, Hkv, d, dtype=bf)
+    fn = getattr(api, which)
+
+    def call(o, lse):
+        if which == "fa_decode_paged_append":
+            fn(q, kn, kn, kp, kp, bt, sl, 0, o, lse)
+        else:
+            fn(q, kp, kp, bt, sl, 0, o, lse)
+
+    good_o = torch.zeros(B, Hq, d, dtype=bf)
+    good_lse = torch.zeros(B, Hq, dtype=torch.float32)
+    for bad_o in (torch.zeros(B, Hq, d // 2, dtype=bf), torch.zeros(B - 1, Hq, d, dtype=bf),
+                  torch.zeros(B, Hq - 1, d, dtype=bf)):
+        with pytest.raises(ValueError, match="o must have shape"):
+            call(bad_o, good_lse)
+    for bad_lse in (torch.zeros(B, Hq - 1, dtype=torch.float32),
+                    torch.zeros(Hq, B, dtype=torch.float32)):
+        with pytest.raises(ValueError, match="lse must have shape"):
+            call(good_o, bad_lse)
+    # right shapes: refused only because these are host tensors
+    with pytest.raises(ValueError, match="CUDA device"):
+        call(good_o, good_lse)

@@ -37,6 +37,37 @@ def test_two_ranks_agree_on_max():
     assert dict(out) == {0: 2.5, 1: 2.5}
 
 
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` outside torchrun re-launches itself under
+    torch.distributed.run with two ranks; with --plumbing (gloo, no kernels)
+    rank 0 prints a line whose n_gpus is 2, and only rank 0 prints."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--plumbing",
+                        "--steps", "3", "--warmup", "3"], capture_output=True, text=True, env=env,
+                       timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["steps"] == 3
+
+
+def test_gpus_flag_must_match_the_launcher():
+    """Under a launcher that set WORLD_SIZE, --gpus must agree with it."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--plumbing"],
+                       capture_output=True, text=True, env=env, timeout=120, cwd=root)
+    assert r.returncode != 0 and "WORLD_SIZE=1" in r.stderr
+
+
 def test_single_rank_is_identity():
     import bench
     assert bench.init_dist(1, "gloo") is None

@@ -7,7 +7,8 @@ import torch
 
 import oracle
 from exact_io_aware_86_b200 import api, inputs
-from parity import BF16_MAX_ABS, BF16_MEAN_ABS, F32_ABS, LSE_ABS, check_bf16, check_close, to_np
+from parity import (BF16_MAX_ABS, BF16_MEAN_ABS, F32_ABS, LSE_ABS, check_bf16, check_bf16_plain,
+                    check_close, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,10 +30,10 @@ def reference(inp):
                                inp.scale)
 
 
-def assert_decode_matches(inp, num_splits):
+def assert_decode_matches(inp, num_splits, plain=False):
     o, lse = run_gpu(inp, num_splits)
     o_ref, lse_ref = reference(inp)
-    check_bf16(o, o_ref, f"O (splits={num_splits})")
+    (check_bf16_plain if plain else check_bf16)(o, o_ref, f"O (splits={num_splits})")
     check_close(lse, lse_ref, LSE_ABS, None, f"LSE (splits={num_splits})")
     return o, lse
 
@@ -46,6 +47,20 @@ CASES = [
     ([4096], 16, 2, 64, 16),
     ([300, 301], 1, 1, 128, 16),
     ([129, 4000, 17], 24, 3, 128, 16),
+    # wide groups: MQA 32:1 and GQA 16:1 (several query tiles per kv head),
+    # 64:1 (eight tiles), 128:1 (two chunks of eight tiles), 12:1 (a ragged tile)
+    ([2000, 33, 0, 517], 32, 1, 128, 16),
+    ([1500, 16, 700], 32, 2, 128, 16),
+    ([900, 65], 64, 1, 128, 64),
+    ([600, 31], 128, 1, 64, 16),
+    ([450, 1, 1000], 36, 3, 128, 16),
+    # page sizes that are not multiples of 16: the per-token gather, stages
+    # that span pages
+    ([1, 2, 17, 300, 1031], 32, 8, 128, 1),
+    ([5, 16, 33, 777], 8, 2, 128, 3),
+    ([8, 9, 640, 2049], 32, 8, 128, 8),
+    ([23, 24, 25, 1000], 16, 4, 64, 24),
+    ([70, 1234], 32, 1, 128, 5),
 ]
 
 
@@ -96,12 +111,46 @@ def test_page_permutation_is_invisible():
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
-def test_unsupported_page_size_is_rejected():
-    inp = inputs.make_decode([40], 4, 1, 128, 8, seed=6103)
+@pytest.mark.parametrize("ps", [1, 2, 3, 8, 24])
+def test_bad_block_table_entry_with_the_per_token_gather(ps):
+    """Page sizes that are not multiples of 16 gather token by token: a used
+    entry outside the pool is read as zeros, never dereferenced, and
+    FA_ERR_DEVICE_BOUNDS is recorded; the other request is exact."""
+    inp = inputs.make_decode([64, 64], 8, 2, 128, ps, seed=6103 + ps)
     q, kp, vp, bt, sl = to_dev(inp)
-    with pytest.raises(api.FAError) as e:
-        api.decode_paged(q, kp, vp, bt, sl, num_splits=1)
-    assert e.value.code == api.FA_ERR_UNSUPPORTED
+    bt[0, 1] = inp.num_pages + 7
+    o, lse = api.decode_paged(q, kp, vp, bt, sl, num_splits=2)
+    assert api.device_error() == api.FA_ERR_DEVICE_BOUNDS
+    assert torch.isfinite(o.float()).all()
+    o_ref, lse_ref = reference(inp)
+    check_bf16(to_np(o)[1:], o_ref[1:], "O, request with valid entries")
+    check_close(to_np(lse)[1:], lse_ref[1:], LSE_ABS, None, "LSE, request with valid entries")
+
+
+def test_empty_pool_and_empty_batch():
+    """num_pages = 0 with every context empty is valid: O = 0 and LSE = -inf,
+    and no page is read (the pool pointer is non-null, its page count 0)."""
+    import ctypes
+    B, Hq, Hkv, d, ps = 3, 8, 2, 128, 16
+    q = torch.randn(B, Hq, d, device="cuda").to(torch.bfloat16)
+    pool = torch.zeros(16, dtype=torch.bfloat16, device="cuda")  # never read
+    bt = torch.full((B, 4), -1, dtype=torch.int32, device="cuda")
+    sl = torch.zeros(B, dtype=torch.int32, device="cuda")
+    lib = api.load_library()
+    for splits in (1, 3, 0):
+        S = splits or api.decode_auto_splits(B, Hq, Hkv, 4, ps)
+        ws = torch.empty(max(api.decode_workspace_size(B, Hq, d, S), 1), dtype=torch.uint8,
+                         device="cuda")
+        o = torch.full((B, Hq, d), 7.0, dtype=torch.bfloat16, device="cuda")
+        lse = torch.zeros(B, Hq, dtype=torch.float32, device="cuda")
+        ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+        st = lib.fa_decode_paged(ptr(q), ptr(pool), ptr(pool), ptr(bt), ptr(sl), ps, splits, ptr(o),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream), B, Hq,
+                                 Hkv, d, 4, 0, 0.0, ptr(lse), ptr(ws), ws.numel())
+        assert st == api.FA_OK
+        assert api.device_error() == api.FA_OK
+        assert torch.count_nonzero(o) == 0
+        assert torch.isneginf(lse).all()
 
 
 def test_bad_block_table_entry_reports_bounds_error():
@@ -147,16 +196,16 @@ def test_fp32_debug_path(ps):
     check_close(to_np(lse), lse_ref, F32_ABS, None, "LSE fp32")
 
 
-# ---- full-size workloads ----------------------------------------------------
+# ---- full-size workloads, checked in full with the plain bounds ------------
 def test_paged_decode_full_size():
     inp = inputs.paged_decode()
-    assert_decode_matches(inp, 0)
+    assert_decode_matches(inp, 0, plain=True)
 
 
 def test_long_decode_full_size():
     inp = inputs.long_decode()
-    o, lse = assert_decode_matches(inp, 0)
+    o, lse = assert_decode_matches(inp, 0, plain=True)
     o1, lse1 = run_gpu(inp, 1)  # one split walks the whole 131072-token context
     o_ref, lse_ref = reference(inp)
-    check_bf16(o1, o_ref, "O one split")
+    check_bf16_plain(o1, o_ref, "O one split")
     check_close(lse1, lse_ref, LSE_ABS, None, "LSE one split")

@@ -13,7 +13,10 @@ output element is at most
 
 plus the bf16 rounding of O (2^-9 |O|).  That bound, computed per element
 from the oracle's exact weights, is the tolerance here; the LSE, which uses
-the unrounded sum, keeps the 1e-3 bound.
+the unrounded sum, keeps the 1e-3 bound.  On the full-size workload the
+bound is evaluated through |v_j - O| <= |v_j| + |O| (the triangle
+inequality), which turns both sums into products with |V| and so needs no
+L x L x d array: a slightly looser bound, still a derived one.
 """
 import numpy as np
 import pytest
@@ -36,7 +39,7 @@ def run(inp):
     return to_np(o), to_np(lse)
 
 
-def check_rows(inp, o, lse, pairs=None):
+def check_rows(inp, o, lse, pairs=None, loose=False):
     qs, ks, vs = inp.meta["descale"]
     q64, k64, v64 = inp.q.double() * qs, inp.k.double() * ks, inp.v.double() * vs
     o_ref, lse_ref = oracle.prefill_fp8(inp.q, inp.k, inp.v, inp.cu_seqlens, inp.causal, inp.scale,
@@ -54,9 +57,18 @@ def check_rows(inp, o, lse, pairs=None):
         P = oracle.prefill_probs(q64, k64, inp.cu_seqlens, inp.causal, inp.scale, b, h, Hkv)
         V = v64[s0:s1, h // (Hq // Hkv)].numpy()                   # [L, d]
         O = o_ref[s0:s1, h]                                         # [L, d]
-        dev = np.abs(V[None, :, :] - O[:, None, :])                 # [L, L, d]
-        bound = (2.0 ** -3 / (1 - 2.0 ** -4)) * np.einsum("ij,ijc->ic", P, dev) \
-            + 2.0 ** -9 * P.max(axis=1, keepdims=True) * dev.sum(axis=1) \
+        if loose:
+            # sum_j w_j |v_j - O| <= (P |V|) + |O|;  sum_j |v_j - O| <= sum_j |v_j| + n |O|
+            # over the visible keys j (where P > 0)
+            vis = (P > 0).astype(np.float64)
+            rel = P @ np.abs(V) + np.abs(O)
+            tot = vis @ np.abs(V) + vis.sum(axis=1, keepdims=True) * np.abs(O)
+        else:
+            dev = np.abs(V[None, :, :] - O[:, None, :])             # [L, L, d]
+            rel = np.einsum("ij,ijc->ic", P, dev)
+            tot = dev.sum(axis=1)
+        bound = (2.0 ** -3 / (1 - 2.0 ** -4)) * rel \
+            + 2.0 ** -9 * P.max(axis=1, keepdims=True) * tot \
             + 2.0 ** -9 * np.abs(O) + 1e-6
         err = np.abs(o[s0:s1, h] - O)
         ratio = (err / bound).max()
@@ -87,12 +99,12 @@ def test_descale_factors():
     check_rows(inp, o, lse)
 
 
-def test_fp8_workload_sampled_pairs():
-    """Causal B=4 H=16 L=2048 d=128 in e4m3: the LSE everywhere, O on four
-    (sequence, head) pairs against the derived bound."""
+def test_fp8_workload_every_pair():
+    """Causal B=4 H=16 L=2048 d=128 in e4m3: the LSE everywhere and O on all
+    64 (sequence, head) pairs, every row, against the derived bound."""
     inp = inputs.fp8_prefill()
     o, lse = run(inp)
-    check_rows(inp, o, lse, pairs=[(0, 0), (1, 7), (2, 15), (3, 3)])
+    check_rows(inp, o, lse, loose=True)
 
 
 def test_rejects_bad_descale_and_head_dim():
