@@ -1,26 +1,39 @@
 """Benchmark of the exact-attention hot path on B200.
 
-One step = one causal MHA prefill (B=4, Hq=Hkv=16, L=2048, d=128, bf16,
-O + LSE) followed by one paged decode (64 requests, Hq=32, Hkv=8, d=128,
-contexts U[1024, 32768] in 16-token pages, split-KV + LSE combine), both
-through the C ABI on inputs already resident in HBM.  Each kernel call is
-timed with CUDA events on the stream it is launched on; a 256 MB buffer is
-written between steps so the prefill inputs (100 MB) never start in L2 (the
-decode's 4.4 GB KV cache exceeds L2 anyway).
+One step = one call of each of the four hot-path workloads, through the C
+ABI on inputs already resident in HBM:
+  - causal MHA prefill, B=4, Hq=Hkv=16, L=2048, d=128, bf16, O + LSE
+    (``parts.prefill``; its TFLOP/s is the line's ``value``);
+  - paged decode, 64 requests, Hq=32, Hkv=8, d=128, contexts
+    U[1024, 32768] in 16-token pages, split-KV + LSE combine
+    (``parts.decode``);
+  - varlen GQA causal prefill, 8 sequences U[512, 8192], Hq=32, Hkv=8
+    (``parts.varlen_gqa_prefill``);
+  - long-context split-KV decode, 2 x 131072 tokens in 64-token pages
+    (``parts.long_decode``).
+Each call is timed with CUDA events on the stream it is launched on, and a
+256 MB buffer is written before every call so no call finds its inputs in
+L2 (the prefill inputs, 100 and 213 MB, are smaller than L2 or close to it;
+the decode caches exceed it anyway).  Per-call times are averaged over the
+--steps timed steps (after --warmup >= 3 untimed ones); the median and the
+minimum are reported beside the mean.
 
-Printed (rank 0, one JSON line): ``value`` = prefill TFLOP/s (causal pairs
-only, 4*d*Hq*L(L+1)/2 per sequence), with the decode's KV GB/s and both
-roofline fractions beside it; ``e2e`` repeats the measurement through the
-public API with pinned host buffers and the host<->device copies inside the
-timed region; ``cpu_baseline`` times the fp64 CPU oracle on a bounded sample.
+Printed (rank 0, one JSON line): ``value`` = causal MHA prefill TFLOP/s
+(causal pairs only, 4*d*Hq*L(L+1)/2 per sequence); every part carries its
+own value and roofline; ``e2e`` repeats the step through the public API
+with pinned host buffers and the host<->device copies inside the timed
+region; ``cpu_baseline`` times the fp64 CPU oracle on a bounded sample of
+each part.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload step|...]
     python bench.py --impl reference ...   # the CPU oracle as the reference arm
 
-Multi-GPU: launched by torch.distributed.run with one rank per GPU, every
-rank runs the same per-GPU workload (weak scaling, no data-path
-collective); the timed region is bracketed by barriers and the max over
-ranks is reported.
+Multi-GPU: one process per GPU.  Under torch.distributed.run (WORLD_SIZE
+set) each rank runs the same per-GPU workload (weak scaling, no data-path
+collective: the parts are independent problems); the timed region is
+bracketed by barriers and the max over ranks is reported.  Without a
+WORLD_SIZE in the environment, --gpus N > 1 re-launches this script under
+torch.distributed.run with N ranks.
 """
 from __future__ import annotations
 
@@ -290,37 +303,54 @@ def oracle_decode_sample(din, n_req: int):
     return decode_bytes(sub), time.perf_counter() - t0
 
 
-def cpu_baseline(pin, din, budget_s: float = 20.0):
+def oracle_sample(inp, n):
+    """Times the oracle on n whole (sequence, head) pairs of a prefill or n
+    whole requests of a decode.  Returns (algorithmic work of the sample:
+    FLOPs or bytes, seconds)."""
+    if isinstance(inp, inputs.PrefillInputs):
+        return oracle_prefill_sample(inp, n)
+    return oracle_decode_sample(inp, n)
+
+
+def cpu_baseline(parts, budget_s: float = 20.0):
+    """The fp64 oracle on a bounded sample of every part of the step (about
+    budget_s seconds in all): whole (sequence, head) pairs of a prefill, whole
+    requests of a decode.  Each part's rate is sample work / sample time;
+    `full_s` is the time the oracle would take on the whole call at that
+    rate (rows and requests are independent, so the rate carries over)."""
     import oracle
     cores = oracle.num_threads()
+    share = budget_s / max(len(parts), 1)
     out = {"kind": "oracle", "cores": cores}
-    if pin is not None:
-        fl, sec = oracle_prefill_sample(pin, 1)
-        n = max(1, min(pin.B * pin.Hq, int((budget_s / 2) / max(sec, 1e-3))))
+    per = {}
+    for p in parts:
+        inp = p.pin if p.is_prefill else p.din
+        total = inp.B * inp.Hq if p.is_prefill else inp.B
+        w, sec = oracle_sample(inp, 1)
+        n = max(1, min(total, int(share / max(sec, 1e-3))))
         if n > 1:
-            fl, sec = oracle_prefill_sample(pin, n)
-        out.update(value=fl / sec / 1e12, unit="TFLOP/s",
-                   sample=f"all rows of {n} of {pin.B * pin.Hq} (sequence, head) pairs of {pin.name}")
-    if din is not None:
-        by, sec = oracle_decode_sample(din, 1)
-        n = max(1, min(din.B, int((budget_s / 2) / max(sec, 1e-3))))
-        if n > 1:
-            by, sec = oracle_decode_sample(din, n)
-        dec = {"value": by / sec / 1e9, "unit": "GB/s",
-               "sample": f"{n} of {din.B} requests (all heads) of {din.name}"}
-        if pin is None:
-            out.update(dec)
-        else:
-            out["decode"] = dec
+            w, sec = oracle_sample(inp, n)
+        rate = w / sec / (1e12 if p.is_prefill else 1e9)
+        what = (f"all rows of {n} of {total} (sequence, head) pairs" if p.is_prefill
+                else f"{n} of {total} requests (all heads)")
+        per[p.key] = {"value": rate, "unit": p.unit, "sample": f"{what} of {inp.name}",
+                      "full_s": round(p.work / (w / sec), 2)}
+    first = per[parts[0].key]
+    out.update(value=first["value"], unit=first["unit"], sample=first["sample"], parts=per)
     return out
 
 
 # --------------------------------------------------------------------------
 # GPU measurement
 # --------------------------------------------------------------------------
+# The default step, in launch order: (workload, key of its entry in "parts")
+STEP = [("mha_prefill", "prefill"), ("paged_decode", "decode"),
+        ("varlen_gqa_prefill", "varlen_gqa_prefill"), ("long_decode", "long_decode")]
+
 WORKLOAD_NAMES = {
     "step": "causal MHA prefill B=4 Hq=Hkv=16 L=2048 d=128 + paged decode 64 req Hq=32 Hkv=8 "
-            "d=128 ctx U[1024,32768] page 16",
+            "d=128 ctx U[1024,32768] page 16 + varlen GQA causal prefill 8 seqs U[512,8192] "
+            "Hq=32 Hkv=8 + split-KV decode 2 x 131072 page 64",
     "mha_prefill": inputs.WORKLOADS["mha_prefill"],
     "varlen_gqa_prefill": inputs.WORKLOADS["varlen_gqa_prefill"],
     "paged_decode": inputs.WORKLOADS["paged_decode"],
@@ -332,39 +362,57 @@ WORKLOAD_NAMES = {
     "fp8_prefill": inputs.WORKLOADS["fp8_prefill"],
 }
 
-
-def make_workload(name):
-    pin = din = None
-    if name in ("step", "mha_prefill"):
-        pin = inputs.mha_prefill()
-    if name == "varlen_gqa_prefill":
-        pin = inputs.varlen_gqa_prefill()
-    if name in ("step", "paged_decode"):
-        din = inputs.paged_decode()
-    if name == "long_decode":
-        din = inputs.long_decode()
-    if name in ("window_prefill", "softcap_prefill", "alibi_prefill", "fp8_prefill"):
-        pin = getattr(inputs, name)()
-    if name == "append_decode":
-        din = inputs.append_decode()
-    return pin, din
+PREFILL_WORKLOADS = ("mha_prefill", "varlen_gqa_prefill", "window_prefill", "softcap_prefill",
+                     "alibi_prefill", "fp8_prefill")
 
 
-class DeviceWorkload:
-    """Device-resident inputs, outputs and scratch for the timed loop."""
+def step_parts(name):
+    """(workload, part key) of each call of a step of `name`."""
+    if name == "step":
+        return list(STEP)
+    return [(name, "prefill" if name in PREFILL_WORKLOADS else "decode")]
 
-    def __init__(self, pin, din, dev):
-        self.pin, self.din = pin, din
-        if pin is not None:
-            self.q, self.k, self.v = (t.to(dev) for t in (pin.q, pin.k, pin.v))
-            self.cu = pin.cu_seqlens.to(dev)
+
+def make_inputs(name):
+    return getattr(inputs, name)()
+
+
+def decode_launches(din, splits: int) -> int:
+    """Kernels one decode call launches: the split kernel, then the LSE
+    combine when a request can have more than one range, the one-CTA plan
+    kernel before them when the batch is too large for the in-kernel plan,
+    and the append + RoPE kernel first for a decode with append."""
+    n = 1
+    if splits > 1:
+        n += 1 + (1 if din.B > api.DECODE_PLAN_MAX_B else 0)
+    return n + (1 if is_append(din) else 0)
+
+
+class Part:
+    """One call of the step: its inputs resident on the device, its outputs
+    and scratch, and its algorithmic work."""
+
+    def __init__(self, workload, key, dev):
+        self.workload, self.key = workload, key
+        inp = make_inputs(workload)
+        self.is_prefill = isinstance(inp, inputs.PrefillInputs)
+        if self.is_prefill:
+            self.pin, self.din = inp, None
+            self.q, self.k, self.v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+            self.cu = inp.cu_seqlens.to(dev)
             self.o = torch.empty(self.q.shape, dtype=torch.bfloat16, device=dev)
-            self.lse = torch.empty(pin.Hq, pin.T, dtype=torch.float32, device=dev)
-            self.max_len = max(pin.lengths)
-            self.variant = variant_of(pin)
+            self.lse = torch.empty(inp.Hq, inp.T, dtype=torch.float32, device=dev)
+            self.max_len = max(inp.lengths)
+            self.variant = variant_of(inp)
             if self.variant.get("alibi_slopes") is not None:
                 self.variant["alibi_slopes"] = self.variant["alibi_slopes"].to(dev)
-        if din is not None:
+            self.work = prefill_flops(inp.lengths, inp.Hq, inp.d, inp.causal,
+                                      self.variant.get("window", (-1, -1)))
+            self.unit = "TFLOP/s"
+            self.launches = 1
+        else:
+            self.pin, self.din = None, inp
+            din = inp
             self.dq, self.kp, self.vp = (t.to(dev) for t in (din.q, din.k_pages, din.v_pages))
             self.bt = din.block_table.to(dev)
             self.sl = (din.cache_seqlens if is_append(din) else din.seq_lens).to(dev)
@@ -382,137 +430,128 @@ class DeviceWorkload:
             self.ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev) if nbytes else None
             self.do = torch.empty_like(self.dq)
             self.dlse = torch.empty(din.B, din.Hq, dtype=torch.float32, device=dev)
+            self.work = decode_bytes(din)
+            self.unit = "GB/s"
+            self.launches = decode_launches(din, self.splits)
 
-    def launches_per_step(self):
-        n = 1 if self.pin is not None else 0
-        if self.din is not None:
-            n += 1 + (2 if self.splits > 1 else 0)  # split kernel (+ plan and combine)
-            n += 1 if is_append(self.din) else 0    # append + RoPE kernel
-        return n
+    @property
+    def name(self):
+        return (self.pin or self.din).name
 
-    def prefill(self):
-        if self.pin.q.dtype == torch.float8_e4m3fn:
-            qs, ks, vs = self.pin.meta["descale"]
-            api.fa_prefill_fp8(self.q, self.k, self.v, self.o, self.lse, self.cu, self.pin.causal,
-                               self.pin.scale, qs, ks, vs, self.max_len)
+    def call(self):
+        if self.is_prefill:
+            pin = self.pin
+            if pin.q.dtype == torch.float8_e4m3fn:
+                qs, ks, vs = pin.meta["descale"]
+                api.fa_prefill_fp8(self.q, self.k, self.v, self.o, self.lse, self.cu, pin.causal,
+                                   pin.scale, qs, ks, vs, self.max_len)
+                return
+            api.fa_prefill(self.q, self.k, self.v, self.o, self.lse, self.cu, pin.causal,
+                           pin.scale, self.max_len, **self.variant)
             return
-        api.fa_prefill(self.q, self.k, self.v, self.o, self.lse, self.cu, self.pin.causal,
-                       self.pin.scale, self.max_len, **self.variant)
-
-    def decode(self):
-        if is_append(self.din):
+        din = self.din
+        if is_append(din):
             # the same slot is rewritten with the same values every call
             api.fa_decode_paged_append(self.dq, self.kn, self.vn, self.kp, self.vp, self.bt,
-                                       self.sl, 0, self.do, self.dlse, self.din.scale, self.cos,
-                                       self.sin, self.din.rotary_dim or None,
-                                       self.din.interleaved, self.ws)
+                                       self.sl, 0, self.do, self.dlse, din.scale, self.cos,
+                                       self.sin, din.rotary_dim or None, din.interleaved, self.ws)
             return
-        api.fa_decode_paged(self.dq, self.kp, self.vp, self.bt, self.sl, 0, self.do,
-                            self.dlse, self.din.scale, self.ws)
+        api.fa_decode_paged(self.dq, self.kp, self.vp, self.bt, self.sl, 0, self.do, self.dlse,
+                            din.scale, self.ws)
+
+    def host_io(self):
+        """(device tensor, pinned host copy) pairs of the inputs the call
+        reads, and of the outputs it writes."""
+        if self.is_prefill:
+            pin = self.pin
+            ins = [(self.q, pin.q), (self.k, pin.k), (self.v, pin.v), (self.cu, pin.cu_seqlens)]
+            outs = [self.o, self.lse]
+        else:
+            din = self.din
+            ins = [(self.dq, din.q), (self.kp, din.k_pages), (self.vp, din.v_pages),
+                   (self.bt, din.block_table),
+                   (self.sl, din.cache_seqlens if is_append(din) else din.seq_lens)]
+            if is_append(din):
+                ins += [(self.kn, din.k_new), (self.vn, din.v_new)]
+                if din.cos is not None:
+                    ins += [(self.cos, din.cos), (self.sin, din.sin)]
+            outs = [self.do, self.dlse]
+        return ([(d, h.pin_memory()) for d, h in ins],
+                [(d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True)) for d in outs])
+
+    def rate(self, ms):
+        """Throughput of one call that took `ms` milliseconds, in self.unit."""
+        return self.work / (ms * 1e-3) / (1e12 if self.is_prefill else 1e9)
 
 
-def time_device(w: DeviceWorkload, steps: int, warmup: int, dist, gpu_index: int):
+def time_device(parts, steps: int, warmup: int, dist, gpu_index: int):
+    """Per-part CUDA-event times (ms lists) over `steps` timed steps, the
+    whole timed region (ms) and the clocks sampled during it."""
     dev = torch.device("cuda", torch.cuda.current_device())
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     for _ in range(warmup):
-        flush.fill_(1.0)
-        if w.pin is not None:
-            w.prefill()
-        if w.din is not None:
-            w.decode()
+        for p in parts:
+            flush.fill_(1.0)
+            p.call()
     torch.cuda.synchronize()
     if api.device_error() != api.FA_OK:
         raise RuntimeError("device error during warm-up")
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in parts] for _ in range(steps)]
     outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     barrier(dist)
     torch.cuda.synchronize()
     with ClockSampler(gpu_index) as clocks:
         outer[0].record()
         for i in range(steps):
-            flush.fill_(float(i))
-            ev[i][0].record()
-            if w.pin is not None:
-                w.prefill()
-            ev[i][1].record()
-            if w.din is not None:
-                w.decode()
-            ev[i][2].record()
+            for j, p in enumerate(parts):
+                flush.fill_(float(i))
+                ev[i][j][0].record()
+                p.call()
+                ev[i][j][1].record()
         outer[1].record()
         torch.cuda.synchronize()
         # keep sampling a little so short regions still get a sample
         time.sleep(0.25)
     barrier(dist)
-    pre = [ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)]
-    dec = [ev[i][1].elapsed_time(ev[i][2]) for i in range(steps)]
+    times = [[ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)]
+             for j in range(len(parts))]
     region = outer[0].elapsed_time(outer[1])
     if api.device_error() != api.FA_OK:
         raise RuntimeError("device error during the timed loop")
-    return pre, dec, region, clocks.summary()
+    return times, region, clocks.summary()
 
 
-def time_e2e(w: DeviceWorkload, steps: int):
-    """Same step through the public API with pinned host inputs: H2D of the
-    step's inputs, the kernels, D2H of the results, all inside the timed
-    region.  Returns (prefill ms list, decode ms list, h2d bytes, d2h bytes)."""
-    pin, din = w.pin, w.din
-    host, h2d, d2h = {}, 0, 0
-    if pin is not None:
-        for n, t in (("q", pin.q), ("k", pin.k), ("v", pin.v), ("cu", pin.cu_seqlens)):
-            host[n] = t.pin_memory()
-            h2d += t.numel() * t.element_size()
-        host["o"] = torch.empty(w.o.shape, dtype=w.o.dtype, pin_memory=True)
-        host["lse"] = torch.empty(w.lse.shape, dtype=w.lse.dtype, pin_memory=True)
-        d2h += w.o.numel() * 2 + w.lse.numel() * 4
-    if din is not None:
-        srcs = [("dq", din.q), ("kp", din.k_pages), ("vp", din.v_pages),
-                ("bt", din.block_table),
-                ("sl", din.cache_seqlens if is_append(din) else din.seq_lens)]
-        if is_append(din):
-            srcs += [("kn", din.k_new), ("vn", din.v_new)]
-            if din.cos is not None:
-                srcs += [("cos", din.cos), ("sin", din.sin)]
-        for n, t in srcs:
-            host[n] = t.pin_memory()
-            h2d += t.numel() * t.element_size()
-        host["do"] = torch.empty(w.do.shape, dtype=w.do.dtype, pin_memory=True)
-        host["dlse"] = torch.empty(w.dlse.shape, dtype=w.dlse.dtype, pin_memory=True)
-        d2h += w.do.numel() * 2 + w.dlse.numel() * 4
-    pre, dec = [], []
-    for i in range(steps + 1):  # first iteration is a warm-up
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        e[0].record()
-        if pin is not None:
-            w.q.copy_(host["q"], non_blocking=True)
-            w.k.copy_(host["k"], non_blocking=True)
-            w.v.copy_(host["v"], non_blocking=True)
-            w.cu.copy_(host["cu"], non_blocking=True)
-            w.prefill()
-            host["o"].copy_(w.o, non_blocking=True)
-            host["lse"].copy_(w.lse, non_blocking=True)
-        e[1].record()
-        if din is not None:
-            w.dq.copy_(host["dq"], non_blocking=True)
-            w.kp.copy_(host["kp"], non_blocking=True)
-            w.vp.copy_(host["vp"], non_blocking=True)
-            w.bt.copy_(host["bt"], non_blocking=True)
-            w.sl.copy_(host["sl"], non_blocking=True)
-            for n in ("kn", "vn", "cos", "sin"):
-                if n in host:
-                    getattr(w, n).copy_(host[n], non_blocking=True)
-            w.decode()
-            host["do"].copy_(w.do, non_blocking=True)
-            host["dlse"].copy_(w.dlse, non_blocking=True)
-        e[2].record()
+def time_e2e(parts, steps: int):
+    """The step through the public API with pinned host buffers: per call,
+    H2D of its inputs, the call, D2H of its results, all inside the timed
+    region.  Returns (per-part ms lists, h2d bytes per step, d2h bytes per
+    step)."""
+    io = [p.host_io() for p in parts]
+    h2d = sum(h.numel() * h.element_size() for ins, _ in io for _, h in ins)
+    d2h = sum(h.numel() * h.element_size() for _, outs in io for _, h in outs)
+    times = [[] for _ in parts]
+    for i in range(steps + 1):  # the first iteration is a warm-up
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in parts]
+        for j, p in enumerate(parts):
+            ins, outs = io[j]
+            ev[j][0].record()
+            for d, h in ins:
+                d.copy_(h, non_blocking=True)
+            p.call()
+            for d, h in outs:
+                h.copy_(d, non_blocking=True)
+            ev[j][1].record()
         torch.cuda.synchronize()
         if i > 0:
-            pre.append(e[0].elapsed_time(e[1]))
-            dec.append(e[1].elapsed_time(e[2]))
-    return pre, dec, h2d, d2h
+            for j in range(len(parts)):
+                times[j].append(ev[j][0].elapsed_time(ev[j][1]))
+    return times, h2d, d2h
 
 
-def roofline(kind, achieved, peak, unit, traffic):
-    return {"bound": "tensor" if kind == "prefill" else "hbm", "achieved": round(achieved, 2),
+def roofline(is_prefill, achieved, peak, unit, traffic):
+    return {"bound": "tensor" if is_prefill else "hbm", "achieved": round(achieved, 2),
             "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic}
 
 
@@ -521,68 +560,59 @@ def run_gpu(args, world, rank, local):
     dist = init_dist(world, "nccl")
     threads = max(1, (os.cpu_count() or 8) // max(world, 1))
     torch.set_num_threads(threads)
-    pin, din = make_workload(args.workload)
+    dev = torch.device("cuda", local)
+    parts = [Part(w, k, dev) for w, k in step_parts(args.workload)]
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        base = cpu_baseline(pin, din, budget_s=args.cpu_budget)
-    w = DeviceWorkload(pin, din, torch.device("cuda", local))
+        base = cpu_baseline(parts, budget_s=args.cpu_budget)
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit() else local
-    pre, dec, region, clocks = time_device(w, args.steps, args.warmup, dist, gpu_index)
+    times, region, clocks = time_device(parts, args.steps, args.warmup, dist, gpu_index)
     e2e_steps = max(2, min(args.steps, args.e2e_steps))
-    epre, edec, h2d, d2h = time_e2e(w, e2e_steps)
+    etimes, h2d, d2h = time_e2e(parts, e2e_steps)
 
     peaks, peak_src = load_peaks()
-    pre_ms = max_over_ranks(dist, statistics.mean(pre) if pin is not None else 0.0, "cuda")
-    dec_ms = max_over_ranks(dist, statistics.mean(dec) if din is not None else 0.0, "cuda")
+    ms = [max_over_ranks(dist, statistics.mean(t), "cuda") for t in times]
+    ems = [max_over_ranks(dist, statistics.mean(t), "cuda") for t in etimes]
     reg_ms = max_over_ranks(dist, region, "cuda")
-    epre_ms = max_over_ranks(dist, statistics.mean(epre) if pin is not None else 0.0, "cuda")
-    edec_ms = max_over_ranks(dist, statistics.mean(edec) if din is not None else 0.0, "cuda")
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
         return
 
-    parts, line = {}, {}
-    if pin is not None:
-        fl = prefill_flops(pin.lengths, pin.Hq, pin.d, pin.causal,
-                           variant_of(pin).get("window", (-1, -1)))
-        tf = world * fl / (pre_ms * 1e-3) / 1e12
-        parts["prefill"] = {
-            "workload": pin.name, "value": round(tf, 2), "unit": "TFLOP/s",
-            "ms": round(pre_ms, 4), "ms_min": round(min(pre), 4), "flops": fl,
+    out_parts = {}
+    for p, t, m in zip(parts, times, ms):
+        rate = world * p.rate(m)
+        if p.is_prefill:
             # an e4m3 contraction takes the fp8 peak: the measured bf16 peak times
             # the nominal fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
-            "roofline": roofline("prefill", tf / world,
-                                 peaks["bf16_tflops"] * (2.0 if is_fp8(pin) else 1.0), "TFLOP/s",
-                                 dram_traffic("prefill", pin.name)),
-            "launches_per_call": 1,
-        }
-    if din is not None:
-        by = decode_bytes(din)
-        gbs = world * by / (dec_ms * 1e-3) / 1e9
-        parts["decode"] = {
-            "workload": din.name, "value": round(gbs, 1), "unit": "GB/s",
-            "ms": round(dec_ms, 4), "ms_min": round(min(dec), 4), "bytes": by,
-            "max_ranges_per_request": w.splits,
-            "workspace_bytes": api.decode_workspace_size(din.B, din.Hq, din.d, w.splits),
-            "roofline": roofline("decode", gbs / world, peaks["hbm_gbs"], "GB/s",
-                                 dram_traffic("decode", din.name)),
-            "launches_per_call": 1 + (2 if w.splits > 1 else 0) + (1 if is_append(din) else 0),
-        }
-    head = parts.get("prefill") or parts.get("decode")
-    dominant = max(parts.values(), key=lambda p: p["ms"])
-    e2e = {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    if pin is not None:
-        e2e.update(value=round(world * parts["prefill"]["flops"] / (epre_ms * 1e-3) / 1e12, 3),
-                   unit="TFLOP/s", ms=round(epre_ms, 3))
-    if din is not None:
-        dv = {"value": round(world * parts["decode"]["bytes"] / (edec_ms * 1e-3) / 1e9, 2),
-              "unit": "GB/s", "ms": round(edec_ms, 3)}
-        if pin is None:
-            e2e.update(dv)
+            peak = peaks["bf16_tflops"] * (2.0 if is_fp8(p.pin) else 1.0)
+            entry = {"workload": p.name, "value": round(rate, 2), "unit": p.unit,
+                     "ms": round(m, 4), "ms_median": round(statistics.median(t), 4),
+                     "ms_min": round(min(t), 4), "flops": p.work,
+                     "roofline": roofline(True, rate / world, peak, "TFLOP/s",
+                                          dram_traffic("prefill", p.name)),
+                     "launches_per_call": p.launches}
         else:
-            e2e["decode"] = dv
+            entry = {"workload": p.name, "value": round(rate, 1), "unit": p.unit,
+                     "ms": round(m, 4), "ms_median": round(statistics.median(t), 4),
+                     "ms_min": round(min(t), 4), "bytes": p.work,
+                     "max_ranges_per_request": p.splits,
+                     "workspace_bytes": api.decode_workspace_size(p.din.B, p.din.Hq, p.din.d,
+                                                                  p.splits),
+                     "roofline": roofline(False, rate / world, peaks["hbm_gbs"], "GB/s",
+                                          dram_traffic("decode", p.name)),
+                     "launches_per_call": p.launches}
+        out_parts[p.key] = entry
+    head_part = parts[0]
+    head = out_parts[head_part.key]
+    dom = max(range(len(parts)), key=lambda j: ms[j])
+    e2e = {"value": round(world * head_part.rate(ems[0]), 3), "unit": head_part.unit,
+           "ms": round(ems[0], 3), "workload": head_part.name,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "parts": {p.key: {"value": round(world * p.rate(m), 3), "unit": p.unit,
+                             "ms": round(m, 3)} for p, m in zip(parts, ems)}}
+    fp8 = any(p.is_prefill and is_fp8(p.pin) for p in parts)
     line = {
         "metric": METRIC,
         "value": head["value"],
@@ -590,21 +620,21 @@ def run_gpu(args, world, rank, local):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(pre_ms + dec_ms, 4),
+        "ms_per_step": round(sum(ms), 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3" if is_fp8(pin) else "bf16",
+        "dtype": "e4m3" if fp8 else "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD_NAMES[args.workload],
-                   "l2": "256 MB buffer written between steps; decode KV (4.4 GB) exceeds L2",
+                   "l2": "256 MB buffer written before every timed call",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
-        "parts": parts,
-        "roofline": dict(dominant["roofline"], kernel=dominant["workload"]),
+        "parts": out_parts,
+        "roofline": dict(out_parts[parts[dom].key]["roofline"], kernel=parts[dom].name),
         "peaks_source": peak_src,
         "region_ms": round(reg_ms, 3),
         "e2e": e2e,
-        "gpu_launches": w.launches_per_step() * args.steps,
+        "gpu_launches": sum(p.launches for p in parts) * args.steps,
         "clocks": clocks,
     }
     if base is not None:
@@ -616,40 +646,33 @@ def run_gpu(args, world, rank, local):
 
 def run_reference(args, world, rank):
     """The reference arm: the fp64 CPU oracle, timed on the host cores on a
-    bounded sample of the same workload; same metric, unit and config."""
+    bounded sample of each call of the same step; same metric, unit and
+    config.  Under torchrun only rank 0 works."""
     if rank != 0:
         return
     import oracle
-    pin, din = make_workload(args.workload)
-    pairs = 1
-    reqs = 2
-    for _ in range(max(0, args.warmup)):
-        if pin is not None:
-            oracle_prefill_sample(pin, pairs)
-        if din is not None:
-            oracle_decode_sample(din, reqs)
-        break  # one warm-up pass is enough for a CPU code path
-    pf, ps, db, ds = 0.0, 0.0, 0.0, 0.0
+    workloads = step_parts(args.workload)
+    ins = [(make_inputs(w), k) for w, k in workloads]
+    pairs, reqs = 1, 2
+    if args.warmup > 0:  # one warm-up pass is enough for a CPU code path
+        for inp, _ in ins:
+            oracle_sample(inp, pairs if isinstance(inp, inputs.PrefillInputs) else reqs)
+    acc = {k: [0.0, 0.0] for _, k in ins}
     for _ in range(args.steps):
-        if pin is not None:
-            f, s = oracle_prefill_sample(pin, pairs)
-            pf, ps = pf + f, ps + s
-        if din is not None:
-            b, s = oracle_decode_sample(din, reqs)
-            db, ds = db + b, ds + s
-    parts = {}
-    if pin is not None:
-        parts["prefill"] = {"workload": pin.name, "value": pf / ps / 1e12, "unit": "TFLOP/s",
-                            "ms": 1e3 * ps / args.steps}
-    if din is not None:
-        parts["decode"] = {"workload": din.name, "value": db / ds / 1e9, "unit": "GB/s",
-                           "ms": 1e3 * ds / args.steps}
-    head = parts.get("prefill") or parts.get("decode")
-    sample = []
-    if pin is not None:
-        sample.append(f"prefill: all rows of {pairs} of {pin.B * pin.Hq} (sequence, head) pairs")
-    if din is not None:
-        sample.append(f"decode: {reqs} of {din.B} requests, all heads")
+        for inp, k in ins:
+            n = pairs if isinstance(inp, inputs.PrefillInputs) else reqs
+            w, sec = oracle_sample(inp, n)
+            acc[k][0] += w
+            acc[k][1] += sec
+    parts, sample = {}, []
+    for inp, k in ins:
+        pre = isinstance(inp, inputs.PrefillInputs)
+        w, sec = acc[k]
+        parts[k] = {"workload": inp.name, "value": w / sec / (1e12 if pre else 1e9),
+                    "unit": "TFLOP/s" if pre else "GB/s", "ms": 1e3 * sec / args.steps}
+        sample.append(f"{inp.name}: all rows of {pairs} of {inp.B * inp.Hq} (sequence, head) pairs"
+                      if pre else f"{inp.name}: {reqs} of {inp.B} requests, all heads")
+    head = parts[ins[0][1]]
     line = {
         "metric": METRIC, "value": head["value"], "unit": head["unit"], "impl": "reference",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -666,7 +689,37 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def relaunch(args, argv):
+    """--gpus N > 1 outside torch.distributed.run: start N ranks of this
+    script under it (127.0.0.1 rendezvous) and return their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd).returncode
+
+
+def run_plumbing(args, world, rank):
+    """--plumbing: the rank and timing plumbing alone on the CPU (gloo), no
+    kernels -- one "step" is a barrier.  Prints the JSON line's rank fields
+    so a CPU test can check a --gpus N launch end to end."""
+    dist = init_dist(world, "gloo")
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        barrier(dist)
+    ms = max_over_ranks(dist, 1e3 * (time.perf_counter() - t0) / max(args.steps, 1), "cpu")
+    if rank == 0:
+        print(json.dumps({"plumbing": True, "n_gpus": world, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step": ms}), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -677,10 +730,21 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plumbing", action="store_true",
+                    help="rank and timing plumbing only, on the CPU (gloo), no kernels")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch(args, argv))
     world, rank, local = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.plumbing:
+        run_plumbing(args, world, rank)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
