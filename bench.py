@@ -11,10 +11,12 @@ ABI on inputs already resident in HBM:
     (``parts.varlen_gqa_prefill``);
   - long-context split-KV decode, 2 x 131072 tokens in 64-token pages
     (``parts.long_decode``).
-Each call is timed with CUDA events on the stream it is launched on, and a
-256 MB buffer is written before every call so no call finds its inputs in
-L2 (the prefill inputs, 100 and 213 MB, are smaller than L2 or close to it;
-the decode caches exceed it anyway).  Per-call times are averaged over the
+Each call is timed with CUDA events on the stream it is launched on.  Before
+every call a 256 MB buffer is written, so no call finds its inputs in L2
+(the prefill inputs, 100 and 213 MB, are smaller than L2 or close to it; the
+decode caches exceed it anyway), and then another 256 MB buffer is read, so
+the dirty lines of that write are written back before the timed call starts
+instead of during it.  Per-call times are averaged over the
 --steps timed steps (after --warmup >= 3 untimed ones); the median and the
 minimum are reported beside the mean.
 
@@ -220,6 +222,19 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+
+    def wait_first(self, timeout: float = 10.0):
+        """Blocks until the sampler has produced a line (nvidia-smi takes a
+        moment to start), so the timed region is sampled from its start."""
+        self.wait_samples(1, timeout)
+
+    def wait_samples(self, n: int, timeout: float = 10.0):
+        if self.proc is None:
+            return
+        base = len(self.lines) if n > 1 else 0
+        t0 = time.time()
+        while len(self.lines) < base + n and time.time() - t0 < timeout:
+            time.sleep(0.02)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -484,14 +499,29 @@ class Part:
         return self.work / (ms * 1e-3) / (1e12 if self.is_prefill else 1e9)
 
 
+class L2Flush:
+    """Writes a buffer larger than L2 (evicting every input), then reads a
+    second one (writing the dirty lines of the first back to memory), so
+    the next call starts with a cold and clean L2."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.float32, device=dev)
+
+    def __call__(self, value: float):
+        self.w.fill_(value)
+        torch.sum(self.r, out=self.acc)
+
+
 def time_device(parts, steps: int, warmup: int, dist, gpu_index: int):
     """Per-part CUDA-event times (ms lists) over `steps` timed steps, the
     whole timed region (ms) and the clocks sampled during it."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     for _ in range(warmup):
         for p in parts:
-            flush.fill_(1.0)
+            flush(1.0)
             p.call()
     torch.cuda.synchronize()
     if api.device_error() != api.FA_OK:
@@ -502,17 +532,18 @@ def time_device(parts, steps: int, warmup: int, dist, gpu_index: int):
     barrier(dist)
     torch.cuda.synchronize()
     with ClockSampler(gpu_index) as clocks:
+        clocks.wait_first()
         outer[0].record()
         for i in range(steps):
             for j, p in enumerate(parts):
-                flush.fill_(float(i))
+                flush(float(i))
                 ev[i][j][0].record()
                 p.call()
                 ev[i][j][1].record()
         outer[1].record()
         torch.cuda.synchronize()
-        # keep sampling a little so short regions still get a sample
-        time.sleep(0.25)
+        # keep sampling a little so short regions still get samples
+        clocks.wait_samples(3)
     barrier(dist)
     times = [[ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)]
              for j in range(len(parts))]
@@ -627,7 +658,8 @@ def run_gpu(args, world, rank, local):
         "dtype": "e4m3" if fp8 else "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD_NAMES[args.workload],
-                   "l2": "256 MB buffer written before every timed call",
+                   "l2": "before every timed call: 256 MB written, then another 256 MB read "
+                         "(cold, clean L2)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "parts": out_parts,
         "roofline": dict(out_parts[parts[dom].key]["roofline"], kernel=parts[dom].name),

@@ -16,12 +16,13 @@
 //   skipped).
 //
 // CTA layout (384 threads = 3 warpgroups, one CTA per SM, persistent):
-//   warp 0      TMA producer: Q tiles once per work item (one barrier pair
-//               per query tile), then K_j, V_j alternately through a ring
-//               of 128 x D smem slots
+//   warp 0      TMA producer of K_j, V_j, alternately through a ring of
+//               128 x D smem slots
 //   warp 1      MMA issuer (converged warp, elected lane) and TMEM owner
 //               (512 columns)
-//   warps 2-3   idle (they complete the first warpgroup)
+//   warp 2      TMA producer of the Q tiles, once per work item, each query
+//               tile on its own barrier pair, refilled as soon as it is free
+//   warp 3      idle (it completes the first warpgroup)
 //   warps 4-7   softmax for query tile 0 (rows q0 .. q0+127)
 //   warps 8-11  softmax for query tile 1 (rows q0+128 .. q0+255)
 // setmaxnreg moves registers from the first warpgroup to the softmax ones.
@@ -91,7 +92,7 @@ constexpr int NQT = 2;            // query tiles per work item
 constexpr int ROWS_PER_ITEM = NQT * BM;
 constexpr int P_CHUNKS = 2;       // P is handed to the P V MMAs in chunks of BN / P_CHUNKS keys
 static_assert(P_CHUNKS == 1 || P_CHUNKS == 2 || P_CHUNKS == 4, "P chunks are whole 32-key quarters");
-constexpr int NUM_WARPS = 12;  // 3 warpgroups: control (producer, MMA, 2 idle), softmax x2
+constexpr int NUM_WARPS = 12;  // 3 warpgroups: control (K/V and Q producers, MMA, 1 idle), softmax x2
 constexpr int NUM_THREADS = NUM_WARPS * 32;
 // Register split between the warpgroups (setmaxnreg).  The launch allots
 // kRegsLaunch per thread; the control group gives most of its share to the
@@ -295,14 +296,6 @@ __device__ __forceinline__ void seq_range(const Params& p, int b, int& start, in
   len = e - s;
 }
 
-// Sum of the four lanes of two packed fp32 pairs.
-__device__ __forceinline__ float sum4(uint64_t a, uint64_t b) {
-  float a0, a1, b0, b1;
-  f2_unpack(a, a0, a1);
-  f2_unpack(b, b0, b1);
-  return (a0 + a1) + (b0 + b1);
-}
-
 __device__ __forceinline__ int blocks_of(int len) { return (len + ROWS_PER_ITEM - 1) / ROWS_PER_ITEM; }
 
 // Work item w -> (b, level, h).  Items are ordered by descending level
@@ -446,12 +439,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort = &sh.abort;
 
   if (warp < 4) {
-    // ---- warpgroup 0: producer (warp 0), MMA issuer (warp 1), warps 2-3 idle ----
+    // ---- warpgroup 0: K/V producer (warp 0), MMA issuer (warp 1), Q producer (warp 2), warp 3 idle ----
     setmaxnreg_dec<kRegsControl>();
    if (warp == 0) {
     // ================ TMA producer (converged warp, elected issue) ================
     {
-      uint32_t kv_it = 0, q_it = 0;
+      uint32_t kv_it = 0;
       for (int it = 0; it < num_items && !*abort; ++it) {
         const int2 item = sh.items[it];
         const int b = item.x, level = item.y >> 16, h = item.y & 0xFFFF;
@@ -460,30 +453,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int q0 = level * ROWS_PER_ITEM;
         int jlo, jhi;
         item_kv_range(p, q0, len, jlo, jhi);
-        const int njobs = jhi - jlo;  // K/V tiles of this item
         const int kh = h / p.group;
-        // K/V tile loads of this item; the first pair goes out before the
-        // wait for the Q buffer, so it overlaps the previous item's tail
-        int next = 0;  // next K/V load (2*j + which) to issue
-        auto issue_kv = [&](int upto) -> bool {
-          for (; next < upto; ++next) {
-            const uint32_t slot = kv_it % C::STAGES;
-            if (!mbar_wait(&sh.kv_empty[slot], ((kv_it / C::STAGES) & 1) ^ 1, abort)) return false;
-            expect_tx_el(&sh.kv_full[slot], C::TILE_BYTES);
-            uint8_t* dst = kv_smem + slot * C::TILE_BYTES;
-            const CUtensorMap* m = (next & 1) ? &tmV : &tmK;
-#pragma unroll
-            for (int pn = 0; pn < C::PANELS; ++pn)
-              tma_load_2d_el(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot],
-                             kh * D + pn * C::PANEL_ELEMS, start + (jlo + (next >> 1)) * BN);
-            ++kv_it;
+        // K/V tiles of this item, 2*j + which; the ring runs on across items,
+        // so the next item's first tiles load while this one drains
+        bool stop = false;
+        for (int next = 0; next < 2 * (jhi - jlo); ++next) {
+          const uint32_t slot = kv_it % C::STAGES;
+          if (!mbar_wait(&sh.kv_empty[slot], ((kv_it / C::STAGES) & 1) ^ 1, abort)) {
+            stop = true;
+            break;
           }
-          return true;
-        };
-        if (!issue_kv(min(2, 2 * njobs))) break;
+          expect_tx_el(&sh.kv_full[slot], C::TILE_BYTES);
+          uint8_t* dst = kv_smem + slot * C::TILE_BYTES;
+          const CUtensorMap* m = (next & 1) ? &tmV : &tmK;
+#pragma unroll
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            tma_load_2d_el(dst + pn * C::PANEL_BYTES, m, &sh.kv_full[slot],
+                           kh * D + pn * C::PANEL_ELEMS, start + (jlo + (next >> 1)) * BN);
+          ++kv_it;
+        }
+        if (stop) break;
+      }
+      // Before the CTA can exit, every load issued must have landed (bounded
+      // wait that ignores the abort flag: the copies finish on their own).
+      for (uint32_t s = 0; s < (uint32_t)C::STAGES && s < kv_it; ++s) {
+        const uint32_t last = kv_it - 1 - ((kv_it - 1 - s) % C::STAGES);  // last use of slot
+        mbar_wait_bounded(&sh.kv_full[last % C::STAGES], (last / C::STAGES) & 1);
+      }
+    }
+   } else if (warp == 2) {
+    // ================ Q producer (converged warp, elected issue) ================
+    // Each query tile's buffer is refilled as soon as the previous item's
+    // last Q K^T of that tile has run (tile 0 usually a step before tile 1),
+    // independently of the K/V ring, so the next item's first Q K^T never
+    // waits behind a K/V slot.
+    {
+      uint32_t q_issued[NQT] = {};
+      for (int it = 0; it < num_items && !*abort; ++it) {
+        const int2 item = sh.items[it];
+        const int b = item.x, level = item.y >> 16, h = item.y & 0xFFFF;
+        int start, len;
+        seq_range(p, b, start, len);
+        const int q0 = level * ROWS_PER_ITEM;
         if (it + 1 < num_items) {
           // the next item's Q tiles come from DRAM; pull them into L2 now so
-          // their load at the next item boundary is short
+          // their load at the next item boundary is short.  (Prefetching the
+          // next item's first K/V tiles as well measured slower.)
           const int2 nx = sh.items[it + 1];
           int ns, nl;
           seq_range(p, nx.x, ns, nl);
@@ -494,30 +509,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int pn = 0; pn < C::PANELS; ++pn)
               tma_prefetch_l2_2d_el(&tmQ, nh * D + pn * C::PANEL_ELEMS, nq0 + t * BM);
         }
-        // each query tile's buffer is refilled as soon as the previous item's
-        // last Q K^T of that tile has run (tile 0 usually a step before tile 1)
         bool stop = false;
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
-          if (!mbar_wait(&sh.q_empty[t], (q_it & 1) ^ 1, abort)) { stop = true; break; }
+          if (!mbar_wait(&sh.q_empty[t], (it & 1) ^ 1, abort)) { stop = true; break; }
           expect_tx_el(&sh.q_full[t], C::TILE_BYTES);
 #pragma unroll
           for (int pn = 0; pn < C::PANELS; ++pn)
             tma_load_2d_el(q_smem + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &sh.q_full[t],
                            h * D + pn * C::PANEL_ELEMS, start + q0 + t * BM);
+          ++q_issued[t];
         }
         if (stop) break;
-        ++q_it;
-        if (!issue_kv(2 * njobs)) break;
       }
-      // Before the CTA can exit, every load issued must have landed (bounded
-      // wait that ignores the abort flag: the copies finish on their own).
-      for (uint32_t s = 0; s < (uint32_t)C::STAGES && s < kv_it; ++s) {
-        const uint32_t last = kv_it - 1 - ((kv_it - 1 - s) % C::STAGES);  // last use of slot
-        mbar_wait_bounded(&sh.kv_full[last % C::STAGES], (last / C::STAGES) & 1);
-      }
-      if (q_it > 0)
-        for (int t = 0; t < NQT; ++t) mbar_wait_bounded(&sh.q_full[t], (q_it - 1) & 1);
+      // every Q load issued must have landed before the CTA exits
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        if (q_issued[t] > 0) mbar_wait_bounded(&sh.q_full[t], (q_issued[t] - 1) & 1);
     }
    } else if (warp == 1) {
     // ================ MMA issuer (converged warp, elected issue) ================
@@ -730,16 +738,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           (GENERAL && p.alibi) ? __ldg(p.alibi + (size_t)b * p.alibi_stride + h) * 1.4426950408889634f
                                : 0.f;
       float m_ref = -INFINITY;
-      // Row sums as interleaved fp32 pairs.  le: the unrounded weights (gives
-      // the LSE).  O is normalised by the sum of the weights the P V MMA
-      // consumed on every tile that needs masking (where rows with few
-      // visible keys live) and by the unrounded weights elsewhere: bf16 keeps
-      // that as le + corr, corr = sum over masked tiles of (rounded -
-      // unrounded), from the per-tile rounded sums lr; e4m3 (whose rounding
-      // is coarser) sums its decoded weights on every tile into lr.
+      // Row sums: le (two interleaved fp32 pairs) = sum of the unrounded
+      // weights, gives the LSE; lr = sum of the rounded (bf16, or decoded
+      // e4m3) weights the P V MMA consumes, normalises O, so O is a weighted
+      // mean with exactly the weights used.
       uint64_t le_a = 0, le_b = 0;
       float lr_a0 = 0.f, lr_a1 = 0.f, lr_b0 = 0.f, lr_b1 = 0.f;
-      float corr = 0.f;
       for (int j = jlo; j < jhi; ++j) {
         if (!mbar_wait(stall ? &sh.stall : &sh.s_full[t], s_phase, abort)) { ok = false; break; }
         stall = false;
@@ -837,7 +841,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t a2 = f2_pack(alpha, alpha);
           le_a = f2_mul(le_a, a2);
           le_b = f2_mul(le_b, a2);
-          corr *= alpha;
           lr_a0 *= alpha;
           lr_a1 *= alpha;
           lr_b0 *= alpha;
@@ -870,18 +873,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t neg2 = f2_pack(-m_use, -m_use);
         // GENERAL: s already holds scaled logits, so the FMA multiplies by 1
         const uint64_t mul2 = GENERAL ? f2_pack(1.f, 1.f) : sl2;
-        // Tiles whose normaliser takes the rounded weights (see the row sums
-        // above): every e4m3 tile, every tile of the mask variants (whose
-        // rows often hold few effective keys), the masked tiles of the plain
-        // kernel.  For bf16 the rounded weights of a quarter are summed from
-        // its packed words after its exponentials, so full tiles run the same
-        // exponential code without that work.
-        const bool round = FP8 || GENERAL || need_mask;
-        float le_tile0 = 0.f;
-        if (!FP8 && round) {
-          le_tile0 = sum4(le_a, le_b);
-          lr_a0 = lr_a1 = lr_b0 = lr_b1 = 0.f;
-        }
         uint32_t e4_lo = 0;  // e4m3: the even pair of a word, waiting for the odd one
         // four 32-key quarters; a chunk is 4 / P_CHUNKS consecutive quarters
         constexpr int QPC = 4 / P_CHUNKS;
@@ -916,7 +907,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               s[c][e >> 1] = pack_bf16x2(p0, p1);
             }
           }
-          if (!FP8 && round) {
+          if constexpr (!FP8) {
+            // the bf16 weights the P V MMA consumes, summed from the packed
+            // words of the quarter (after its exponentials)
 #pragma unroll
             for (int w = 0; w < 16; w += 2) {
               lr_a0 = add_bf16lo_f32(s[c][w], lr_a0);
@@ -940,10 +933,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_st16(s_col + c * 16, s[c]);
         }
         if (QPC == 4 && rescale) rescale_o();
-        // bf16: the normaliser takes this tile's rounded weights:
-        // corr += sum(rounded) - sum(unrounded) over the tile
-        if (!FP8 && round)
-          corr += ((lr_a0 + lr_a1) + (lr_b0 + lr_b1)) - (sum4(le_a, le_b) - le_tile0);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sh.p_full[t][P_CHUNKS - 1]);
@@ -957,7 +946,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       f2_unpack(le_a, la0, la1);
       f2_unpack(le_b, lb0, lb1);
       const float l_exact = (la0 + la1) + (lb0 + lb1);
-      const float l_norm = FP8 ? (lr_a0 + lr_a1) + (lr_b0 + lr_b1) : l_exact + corr;
+      const float l_norm = (lr_a0 + lr_a1) + (lr_b0 + lr_b1);
       const bool valid = qpos < len;
       const float inv_l = p.o_scale / l_norm;
       const size_t grow = (size_t)(start + qpos);
