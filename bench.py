@@ -504,14 +504,14 @@ class L2Flush:
     second one (writing the dirty lines of the first back to memory), so
     the next call starts with a cold and clean L2."""
 
-    def __init__(self, dev):
-        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    def __init__(self, dev, nbytes: int = L2_FLUSH_BYTES):
+        self.w = torch.empty(nbytes // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(nbytes // 4, dtype=torch.float32, device=dev)
         self.acc = torch.zeros((), dtype=torch.float32, device=dev)
 
     def __call__(self, value: float):
         self.w.fill_(value)
-        torch.sum(self.r, out=self.acc)
+        torch.sum(self.r, dim=0, out=self.acc)
 
 
 def time_device(parts, steps: int, warmup: int, dist, gpu_index: int):

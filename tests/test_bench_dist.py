@@ -123,3 +123,16 @@ def test_append_decode_bytes():
     pages = 1 + 3
     extra = 2 * (2 * 2 * 2 * 16 * 2) + 2 * 2 * 4 * 4
     assert bench.decode_bytes(a) == kv + qo + 4 * pages + 4 * 2 + extra
+
+
+def test_l2_flush_writes_then_reads():
+    """The benchmark's flush writes one buffer and reads another (so the
+    dirty lines of the write are gone before a timed call); checked on a
+    small CPU buffer."""
+    import torch
+    import bench
+    f = bench.L2Flush(torch.device("cpu"), 1 << 16)
+    f.r.fill_(0.5)
+    f(3.0)
+    assert float(f.w.min()) == 3.0 and float(f.w.max()) == 3.0
+    assert float(f.acc) == 0.5 * f.r.numel()
