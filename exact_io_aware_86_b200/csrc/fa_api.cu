@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "fa.h"
 #include "ptx.cuh"
@@ -112,6 +113,28 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kMaxDevices = 64;
 
+// Launches `kernel` with programmatic stream serialization: it may start
+// while the stream's previous kernel drains, and must itself execute
+// griddepcontrol.wait before it reads or writes global memory that kernel
+// could touch.
+template <typename... KArgs, typename... Args>
+fa_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem,
+                     cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? FA_OK
+                                                                                      : FA_ERR_CUDA;
+}
+
 // Launch set-up of one kernel: the dynamic shared-memory limit is an
 // attribute of the kernel on a device, so it is set once per device (under a
 // lock, as several host threads may launch on several devices), together
@@ -206,6 +229,8 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   // split only fits if the launch allots kRegsLaunch registers per thread
   // (otherwise setmaxnreg.inc could never be satisfied).
   if (launch_regs < (int)kRegsLaunch) return FA_ERR_UNSUPPORTED;
+  // (A programmatic dependent launch, to overlap the set-up with the
+  // stream's previous kernel, measured no faster.)
   prefill_kernel<D, GENERAL, FP8><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -338,18 +363,9 @@ fa_status launch_decode(const void* q, const void* kp, const void* vp, const int
   if (split) {
     // a programmatic dependent of the split kernel: its CTAs are scheduled
     // while the split kernel drains and wait for it to complete
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)(B * Hq));
-    cfg.blockDim = dim3(COMBINE_WARPS * 32);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = grid > 0 ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, combine_kernel<D>, p) != cudaSuccess) return FA_ERR_CUDA;
+    const fa_status st = launch_pdl(combine_kernel<D>, dim3((unsigned)(B * Hq)),
+                                    dim3(COMBINE_WARPS * 32), 0, stream, p);
+    if (st != FA_OK) return st;
   }
   return FA_OK;
 }
