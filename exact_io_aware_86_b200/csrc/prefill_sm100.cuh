@@ -105,7 +105,7 @@ static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= NUM_THREADS * kRegsLaun
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int MAX_LEVELS = 4096;  // max_seqlen <= 4096 * 256
-constexpr int MAX_ITEMS_PER_CTA = 192;
+constexpr int MAX_ITEMS_PER_CTA = 96;
 constexpr int SMEM_LIMIT = 232448;  // dynamic shared memory per CTA on sm_100
 
 // Instruction descriptor for e4m3 x e4m3 -> fp32 (kind::f8f6f4): the A and
@@ -217,11 +217,12 @@ struct Shared {
   uint64_t s_full[NQT], o_full[NQT];
   uint64_t p_full[NQT][P_CHUNKS];  // one chunk of P written to TMEM
   uint64_t stall;                  // never arrived at (timeout test hook)
+  uint64_t q_issued;               // the first item's Q loads have been issued
   uint32_t tmem_base;
   int abort;
   int num_items;                     // items this CTA processes
   int total_items;
-  int2 items[MAX_ITEMS_PER_CTA];     // (b, level << 16 | h)
+  int4 items[MAX_ITEMS_PER_CTA];     // (start, len, level << 16 | h, b)
 };
 
 // Work-list construction scratch; only live before the main loop, so it
@@ -359,6 +360,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(&sh.mma_done, 1);
     mbar_init(&sh.stall, 1);
+    mbar_init(&sh.q_issued, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&sh.kv_full[s], 1);
       mbar_init(&sh.kv_empty[s], 1);
@@ -424,9 +426,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   for (int i = tid; i < sh.num_items; i += NUM_THREADS) {
     const int G = gridDim.x, c = blockIdx.x;
     const int w = i * G + ((i & 1) ? (G - 1 - c) : c);
-    int b, level, h;
+    int b, level, h, st, len;
     decode_item(p, ps, w, b, level, h);
-    sh.items[i] = make_int2(b, (level << 16) | h);
+    seq_range(p, b, st, len);
+    // the sequence range travels with the item: no role reads cu_seqlens
+    // (global memory) at an item boundary
+    sh.items[i] = make_int4(st, len, (level << 16) | h, b);
   }
   // the plan scratch was written through the generic proxy; the ring's TMA
   // loads (async proxy) overwrite it after the barrier below
@@ -446,10 +451,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     {
       uint32_t kv_it = 0;
       for (int it = 0; it < num_items && !*abort; ++it) {
-        const int2 item = sh.items[it];
-        const int b = item.x, level = item.y >> 16, h = item.y & 0xFFFF;
-        int start, len;
-        seq_range(p, b, start, len);
+        const int4 item = sh.items[it];
+        const int start = item.x, len = item.y, level = item.z >> 16, h = item.z & 0xFFFF;
         const int q0 = level * ROWS_PER_ITEM;
         int jlo, jhi;
         item_kv_range(p, q0, len, jlo, jhi);
@@ -460,6 +463,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int next = 0; next < 2 * (jhi - jlo); ++next) {
           const uint32_t slot = kv_it % C::STAGES;
           if (!mbar_wait(&sh.kv_empty[slot], ((kv_it / C::STAGES) & 1) ^ 1, abort)) {
+            stop = true;
+            break;
+          }
+          // At the start every CTA loads at once: the first K tile goes out,
+          // then the rest of the ring waits until the first item's Q tiles
+          // are issued, so the loads the first Q K^T needs come first.
+          if (kv_it == 1 && !mbar_wait(&sh.q_issued, 0, abort)) {
             stop = true;
             break;
           }
@@ -490,25 +500,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     {
       uint32_t q_issued[NQT] = {};
       for (int it = 0; it < num_items && !*abort; ++it) {
-        const int2 item = sh.items[it];
-        const int b = item.x, level = item.y >> 16, h = item.y & 0xFFFF;
-        int start, len;
-        seq_range(p, b, start, len);
+        const int4 item = sh.items[it];
+        const int start = item.x, level = item.z >> 16, h = item.z & 0xFFFF;
         const int q0 = level * ROWS_PER_ITEM;
-        if (it + 1 < num_items) {
-          // the next item's Q tiles come from DRAM; pull them into L2 now so
-          // their load at the next item boundary is short.  (Prefetching the
-          // next item's first K/V tiles as well measured slower.)
-          const int2 nx = sh.items[it + 1];
-          int ns, nl;
-          seq_range(p, nx.x, ns, nl);
-          const int nq0 = ns + (nx.y >> 16) * ROWS_PER_ITEM, nh = nx.y & 0xFFFF;
-#pragma unroll
-          for (int t = 0; t < NQT; ++t)
-#pragma unroll
-            for (int pn = 0; pn < C::PANELS; ++pn)
-              tma_prefetch_l2_2d_el(&tmQ, nh * D + pn * C::PANEL_ELEMS, nq0 + t * BM);
-        }
         bool stop = false;
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
@@ -521,6 +515,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ++q_issued[t];
         }
         if (stop) break;
+        if (it == 0) {
+          // the K/V ring may now fill; the first prefetch below waits until
+          // this item's Q has landed, so it never delays the first loads
+          if (lane == 0) mbar_arrive(&sh.q_issued);
+          __syncwarp();
+          if (!mbar_wait(&sh.q_full[NQT - 1], 0, abort)) break;
+        }
+        if (it + 1 < num_items) {
+          // the next item's Q tiles come from DRAM; pull them into L2 now so
+          // their load at the next item boundary is short.  (Prefetching the
+          // next item's first K/V tiles as well measured slower.)
+          const int4 nx = sh.items[it + 1];
+          const int nq0 = nx.x + (nx.z >> 16) * ROWS_PER_ITEM, nh = nx.z & 0xFFFF;
+#pragma unroll
+          for (int t = 0; t < NQT; ++t)
+#pragma unroll
+            for (int pn = 0; pn < C::PANELS; ++pn)
+              tma_prefetch_l2_2d_el(&tmQ, nh * D + pn * C::PANEL_ELEMS, nq0 + t * BM);
+        }
       }
       // every Q load issued must have landed before the CTA exits
 #pragma unroll
@@ -576,11 +589,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // longer softmax it measured slower.
       bool la_done = false;  // this item's first tile-0 S was issued by the lookahead
       for (int it = 0; it < num_items && ok; ++it) {
-        const int2 item = sh.items[it];
-        const int b = item.x, level = item.y >> 16;
-        int start, len;
-        seq_range(p, b, start, len);
-        (void)start;
+        const int4 item = sh.items[it];
+        const int len = item.y, level = item.z >> 16;
         const int q0 = level * ROWS_PER_ITEM;
         // K/V tile range of each query tile; an absent second tile gets an
         // empty range
@@ -641,12 +651,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             s0_last = j == hi0 - 1;
             qr0 = qr0 || s0_last;
           } else if (!GENERAL && j == jhi && hi0 < jhi && qr0 && it + 1 < num_items) {
-            const int2 nx = sh.items[it + 1];
-            int ns, nl;
-            seq_range(p, nx.x, ns, nl);
-            (void)ns;
+            const int4 nx = sh.items[it + 1];
             int nlo, nhi;
-            tile_kv_range(p, (nx.y >> 16) * ROWS_PER_ITEM, nl, nlo, nhi);
+            tile_kv_range(p, (nx.z >> 16) * ROWS_PER_ITEM, nx.y, nlo, nhi);
             if (nhi > nlo) {
               const uint32_t nk = base + 2 * (jhi - jlo);  // the next item's first K
               if (!mbar_wait(&sh.q_full[0], (it + 1) & 1, abort) ||
@@ -724,10 +731,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint64_t sl2 = f2_pack(sl, sl);
     bool ok = true;
     for (int it = 0; it < num_items && ok; ++it) {
-      const int2 item = sh.items[it];
-      const int b = item.x, level = item.y >> 16, h = item.y & 0xFFFF;
-      int start, len;
-      seq_range(p, b, start, len);
+      const int4 item = sh.items[it];
+      const int start = item.x, len = item.y, level = item.z >> 16, h = item.z & 0xFFFF, b = item.w;
       const int rs = level * ROWS_PER_ITEM + t * BM;  // first row of this tile
       if (rs >= len) continue;
       int jlo, jhi;
