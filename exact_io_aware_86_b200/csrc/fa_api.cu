@@ -173,7 +173,7 @@ struct Variant {
   bool general() const { return softcap > 0.f || alibi != nullptr || wl >= 0 || wr > 0; }
 };
 
-template <int D, bool GENERAL, bool FP8 = false>
+template <int D, bool GENERAL, bool FP8 = false, bool LOGIT = false>
 fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                          const int32_t* cu, int B, int Hq, int Hkv, int causal, float scale,
                          cudaStream_t stream, int T, int max_seqlen, const Variant& var,
@@ -224,14 +224,14 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   const int smem = smem_bytes<D, FP8>();
   static KernelSetup setup;
   int launch_regs = 0;
-  if (!setup_kernel(setup, prefill_kernel<D, GENERAL, FP8>, smem, &launch_regs)) return FA_ERR_CUDA;
+  if (!setup_kernel(setup, prefill_kernel<D, GENERAL, FP8, LOGIT>, smem, &launch_regs)) return FA_ERR_CUDA;
   // The kernel hands registers between its warpgroups with setmaxnreg; the
   // split only fits if the launch allots kRegsLaunch registers per thread
   // (otherwise setmaxnreg.inc could never be satisfied).
   if (launch_regs < (int)kRegsLaunch) return FA_ERR_UNSUPPORTED;
   // (A programmatic dependent launch, to overlap the set-up with the
   // stream's previous kernel, measured no faster.)
-  prefill_kernel<D, GENERAL, FP8><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, GENERAL, FP8, LOGIT><<<(unsigned)grid, NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -404,16 +404,28 @@ fa_status fa_prefill_ex(const void* q, const void* k, const void* v, void* o, fl
     return FA_ERR_UNSUPPORTED;
   if (B == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // three kernels per head size: plain causal / full, a band mask alone,
+  // and a band with softcap or ALiBi
   const bool gen = var.general();
-  if (d == 64)
-    return gen ? launch_prefill<64, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
-                                          s, total_tokens, max_seqlen, var)
-               : launch_prefill<64, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
-                                           scale, s, total_tokens, max_seqlen, var);
-  return gen ? launch_prefill<128, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
-                                         s, total_tokens, max_seqlen, var)
-             : launch_prefill<128, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
-                                          s, total_tokens, max_seqlen, var);
+  const bool logit = var.softcap > 0.f || var.alibi != nullptr;
+  if (d == 64) {
+    if (!gen)
+      return launch_prefill<64, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
+                                       total_tokens, max_seqlen, var);
+    return logit ? launch_prefill<64, true, false, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv,
+                                                         causal, scale, s, total_tokens,
+                                                         max_seqlen, var)
+                 : launch_prefill<64, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
+                                            s, total_tokens, max_seqlen, var);
+  }
+  if (!gen)
+    return launch_prefill<128, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
+                                      total_tokens, max_seqlen, var);
+  return logit ? launch_prefill<128, true, false, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv,
+                                                        causal, scale, s, total_tokens, max_seqlen,
+                                                        var)
+               : launch_prefill<128, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
+                                           total_tokens, max_seqlen, var);
 }
 
 fa_status fa_prefill_fp8(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -57,9 +57,11 @@
 // The row max is taken over the first two 32-column loads of S while the last
 // two are still in flight.
 //
-// Mask variants ("flash-attention" skill page, section 3.3), compiled into a
-// second instantiation (GENERAL = true) so the plain causal / full kernel
-// keeps its lean inner loop:
+// Mask variants ("flash-attention" skill page, section 3.3), compiled into
+// instantiations of their own (GENERAL = true) so the plain causal / full
+// kernel keeps its lean inner loop; LOGIT = true adds the softcap and ALiBi
+// passes over the scores, and a band alone (LOGIT = false) scales its scores
+// like the plain kernel, inside the exponent's FMA:
 //   - sliding window (left, right): query i sees keys i-left .. i+right.
 //     Each query tile visits only the K/V tiles that intersect its band
 //     [lo, hi), so a long sequence costs O(L * window), not O(L^2);
@@ -330,13 +332,14 @@ __device__ void decode_item(const Params& p, const PlanScratch& sh, int w, int& 
   }
 }
 
-template <int D, bool GENERAL, bool FP8 = false>
+template <int D, bool GENERAL, bool FP8 = false, bool LOGIT = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV,
                    const Params p) {
   using C = Cfg<D, FP8>;
   static_assert(!(GENERAL && FP8), "mask variants are not built for e4m3");
+  static_assert(GENERAL || !LOGIT, "softcap and ALiBi come with the mask-variant kernel");
   // one exp2 pair in POLY_EVERY on the FMA pipe, the rest on MUFU (0: all MUFU)
   constexpr int POLY_EVERY = 0;
   extern __shared__ uint8_t smem_raw[];
@@ -738,9 +741,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int jlo, jhi;
       tile_kv_range(p, rs, len, jlo, jhi);
       const int qpos = rs + row;
-      // ALiBi slope of this (sequence, head) in log2 units (GENERAL only)
+      // ALiBi slope of this (sequence, head) in log2 units (LOGIT only)
       const float slope2 =
-          (GENERAL && p.alibi) ? __ldg(p.alibi + (size_t)b * p.alibi_stride + h) * 1.4426950408889634f
+          (LOGIT && p.alibi) ? __ldg(p.alibi + (size_t)b * p.alibi_stride + h) * 1.4426950408889634f
                                : 0.f;
       float m_ref = -INFINITY;
       // Row sums: le (two interleaved fp32 pairs) = sum of the unrounded
@@ -770,10 +773,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           need_mask = kv0 + BN > len || (p.causal && kv0 + BN - 1 > rs);
           lim_hi = min(len, p.causal ? qpos + 1 : len) - kv0;
         }
-        // GENERAL: logits in log2 units (optional cap, then the ALiBi
-        // penalty), then the band mask; plain: the mask only
+        // softcap or ALiBi: logits in log2 units (optional cap, then the
+        // ALiBi penalty); then the mask (band, sequence end, causal)
         auto prepare = [&](uint32_t (&x)[32], int c) {
-          if constexpr (GENERAL) {
+          if constexpr (LOGIT) {
             if (p.cap_out > 0.f) {
 #pragma unroll
               for (int e = 0; e < 32; ++e)
@@ -826,7 +829,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         prepare(s[3], 3);
         chunk_max(s[2], s[3], mx + 4);
         const float mx_s = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
-                                 fmaxf(mx[6], mx[7])) * (GENERAL ? 1.f : sl);
+                                 fmaxf(mx[6], mx[7])) * (LOGIT ? 1.f : sl);
         // Lazy rescale, decided per row: the reference max moves only when the
         // tile max exceeds it by more than the threshold.  The exponentials
         // start at once with this row's reference; O is rescaled in tensor
@@ -876,8 +879,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // s[c][0..] in order
         const float m_use = (GENERAL && m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t neg2 = f2_pack(-m_use, -m_use);
-        // GENERAL: s already holds scaled logits, so the FMA multiplies by 1
-        const uint64_t mul2 = GENERAL ? f2_pack(1.f, 1.f) : sl2;
+        // LOGIT: s already holds scaled logits, so the FMA multiplies by 1
+        const uint64_t mul2 = LOGIT ? f2_pack(1.f, 1.f) : sl2;
         uint32_t e4_lo = 0;  // e4m3: the even pair of a word, waiting for the odd one
         // four 32-key quarters; a chunk is 4 / P_CHUNKS consecutive quarters
         constexpr int QPC = 4 / P_CHUNKS;

@@ -49,11 +49,14 @@ def test_prefill_wait_times_out_then_recovers(causal):
     check_close(to_np(lse), lse_ref, LSE_ABS, None, "LSE after the timeout")
 
 
-def test_prefill_variant_wait_times_out_then_recovers():
-    """The mask-variant instantiation takes the same path."""
+@pytest.mark.parametrize("softcap", [0.0, 20.0])
+def test_prefill_variant_wait_times_out_then_recovers(softcap):
+    """The mask-variant instantiations (a band alone; a band with softcap)
+    take the same path."""
     inp = inputs.make_prefill([600, 77], 4, 4, 128, True, seed=8002)
     q, k, v, cu = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.cu_seqlens))
-    run = lambda: api.prefill(q, k, v, cu, causal=True, scale=inp.scale, window=(100, 0))
+    run = lambda: api.prefill(q, k, v, cu, causal=True, scale=inp.scale, window=(100, 0),
+                              softcap=softcap)
     run()
     assert api.device_error() == api.FA_OK
     code, dt = _with_stall(api.STALL_PREFILL, run)
@@ -61,7 +64,7 @@ def test_prefill_variant_wait_times_out_then_recovers():
     o, lse = run()
     assert api.device_error() == api.FA_OK
     o_ref, lse_ref = oracle.prefill(inp.q, inp.k, inp.v, inp.cu_seqlens, True, inp.scale,
-                                    window=(100, 0))
+                                    window=(100, 0), softcap=softcap)
     check_bf16(to_np(o), o_ref, "O after the timeout")
 
 
