@@ -173,7 +173,7 @@ struct Variant {
   bool general() const { return softcap > 0.f || alibi != nullptr || wl >= 0 || wr > 0; }
 };
 
-template <int D, bool GENERAL, bool FP8 = false, bool LOGIT = false>
+template <int D, bool GENERAL, bool FP8 = false, int LOGIT = 0>
 fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
                          const int32_t* cu, int B, int Hq, int Hkv, int causal, float scale,
                          cudaStream_t stream, int T, int max_seqlen, const Variant& var,
@@ -404,28 +404,37 @@ fa_status fa_prefill_ex(const void* q, const void* k, const void* v, void* o, fl
     return FA_ERR_UNSUPPORTED;
   if (B == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // three kernels per head size: plain causal / full, a band mask alone,
-  // and a band with softcap or ALiBi
+  // four kernels per head size: plain causal / full; a band mask alone;
+  // causal ALiBi (no softcap), whose penalty is linear in the key; and a
+  // band with softcap and / or ALiBi, rewriting every score
   const bool gen = var.general();
-  const bool logit = var.softcap > 0.f || var.alibi != nullptr;
+  const int logit = (var.softcap > 0.f || var.alibi != nullptr)
+                        ? ((var.alibi != nullptr && var.softcap == 0.f && var.wr == 0) ? 2 : 1)
+                        : 0;
   if (d == 64) {
     if (!gen)
       return launch_prefill<64, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
                                        total_tokens, max_seqlen, var);
-    return logit ? launch_prefill<64, true, false, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv,
-                                                         causal, scale, s, total_tokens,
-                                                         max_seqlen, var)
-                 : launch_prefill<64, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale,
-                                            s, total_tokens, max_seqlen, var);
+    if (logit == 1)
+      return launch_prefill<64, true, false, 1>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
+                                                scale, s, total_tokens, max_seqlen, var);
+    if (logit == 2)
+      return launch_prefill<64, true, false, 2>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
+                                                scale, s, total_tokens, max_seqlen, var);
+    return launch_prefill<64, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
+                                    total_tokens, max_seqlen, var);
   }
   if (!gen)
     return launch_prefill<128, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
                                       total_tokens, max_seqlen, var);
-  return logit ? launch_prefill<128, true, false, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv,
-                                                        causal, scale, s, total_tokens, max_seqlen,
-                                                        var)
-               : launch_prefill<128, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
-                                           total_tokens, max_seqlen, var);
+  if (logit == 1)
+    return launch_prefill<128, true, false, 1>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
+                                               scale, s, total_tokens, max_seqlen, var);
+  if (logit == 2)
+    return launch_prefill<128, true, false, 2>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
+                                               scale, s, total_tokens, max_seqlen, var);
+  return launch_prefill<128, true>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
+                                   total_tokens, max_seqlen, var);
 }
 
 fa_status fa_prefill_fp8(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -59,9 +59,12 @@
 //
 // Mask variants ("flash-attention" skill page, section 3.3), compiled into
 // instantiations of their own (GENERAL = true) so the plain causal / full
-// kernel keeps its lean inner loop; LOGIT = true adds the softcap and ALiBi
-// passes over the scores, and a band alone (LOGIT = false) scales its scores
-// like the plain kernel, inside the exponent's FMA:
+// kernel keeps its lean inner loop.  LOGIT selects how the scores reach the
+// exponent: 0 (a band alone) scales them like the plain kernel, inside the
+// exponent's FMA; 1 rewrites every score in place (softcap, then ALiBi);
+// 2 is ALiBi without softcap under a right bound of 0, where every visible
+// key precedes its query, so the penalty slope * (key - query) is linear in
+// the key's column and joins the row max and the exponent's FMA:
 //   - sliding window (left, right): query i sees keys i-left .. i+right.
 //     Each query tile visits only the K/V tiles that intersect its band
 //     [lo, hi), so a long sequence costs O(L * window), not O(L^2);
@@ -332,14 +335,16 @@ __device__ void decode_item(const Params& p, const PlanScratch& sh, int w, int& 
   }
 }
 
-template <int D, bool GENERAL, bool FP8 = false, bool LOGIT = false>
+template <int D, bool GENERAL, bool FP8 = false, int LOGIT = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV,
                    const Params p) {
   using C = Cfg<D, FP8>;
   static_assert(!(GENERAL && FP8), "mask variants are not built for e4m3");
-  static_assert(GENERAL || !LOGIT, "softcap and ALiBi come with the mask-variant kernel");
+  static_assert(GENERAL || LOGIT == 0, "softcap and ALiBi come with the mask-variant kernel");
+  constexpr bool INPLACE = LOGIT == 1;  // scores rewritten in place
+  constexpr bool LINEAR = LOGIT == 2;   // causal ALiBi folded into max and exponent
   // one exp2 pair in POLY_EVERY on the FMA pipe, the rest on MUFU (0: all MUFU)
   constexpr int POLY_EVERY = 0;
   extern __shared__ uint8_t smem_raw[];
@@ -741,9 +746,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int jlo, jhi;
       tile_kv_range(p, rs, len, jlo, jhi);
       const int qpos = rs + row;
-      // ALiBi slope of this (sequence, head) in log2 units (LOGIT only)
+      // ALiBi slope of this (sequence, head) in log2 units (LOGIT 1 and 2)
       const float slope2 =
-          (LOGIT && p.alibi) ? __ldg(p.alibi + (size_t)b * p.alibi_stride + h) * 1.4426950408889634f
+          (LOGIT != 0 && p.alibi) ? __ldg(p.alibi + (size_t)b * p.alibi_stride + h) * 1.4426950408889634f
                                : 0.f;
       float m_ref = -INFINITY;
       // Row sums: le (two interleaved fp32 pairs) = sum of the unrounded
@@ -776,7 +781,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // softcap or ALiBi: logits in log2 units (optional cap, then the
         // ALiBi penalty); then the mask (band, sequence end, causal)
         auto prepare = [&](uint32_t (&x)[32], int c) {
-          if constexpr (LOGIT) {
+          if constexpr (INPLACE) {
             if (p.cap_out > 0.f) {
 #pragma unroll
               for (int e = 0; e < 32; ++e)
@@ -803,15 +808,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // row max: four independent chains of three-input maxima per pair of
         // chunks; the max of chunks 0-1 runs while chunks 2-3 load
         float mx[8];
-        auto chunk_max = [&](const uint32_t (&a)[32], const uint32_t (&b)[32], float* m) {
+        // LINEAR: the max of s * scale + slope * column (log2 units); the row's
+        // constant slope * (kv0 - query) is added once below
+        const uint64_t sp2 = f2_pack(slope2, slope2);
+        auto chunk_max = [&](const uint32_t (&a)[32], const uint32_t (&b)[32], float* m, int cb) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t* src = (k < 2) ? a : b;
             const int o = (k & 1) * 16;
-            m[k] = fmaxf(__uint_as_float(src[o]), __uint_as_float(src[o + 1]));
+            if constexpr (LINEAR) {
+              const int c0 = cb + (k >> 1) * 32 + o;  // column of src[o]
+              float y[16];
 #pragma unroll
-            for (int e = 2; e < 16; e += 2)
-              m[k] = fmax3(m[k], __uint_as_float(src[o + e]), __uint_as_float(src[o + e + 1]));
+              for (int e = 0; e < 16; e += 2) {
+                const uint64_t t = f2_mul(sp2, f2_pack((float)(c0 + e), (float)(c0 + e + 1)));
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(src[o + e]), __uint_as_float(src[o + e + 1])),
+                                 sl2, t),
+                          y[e], y[e + 1]);
+              }
+              m[k] = fmaxf(y[0], y[1]);
+#pragma unroll
+              for (int e = 2; e < 16; e += 2) m[k] = fmax3(m[k], y[e], y[e + 1]);
+            } else {
+              m[k] = fmaxf(__uint_as_float(src[o]), __uint_as_float(src[o + 1]));
+#pragma unroll
+              for (int e = 2; e < 16; e += 2)
+                m[k] = fmax3(m[k], __uint_as_float(src[o + e]), __uint_as_float(src[o + e + 1]));
+            }
           }
         };
         tmem_ld32(s_col, s[0]);
@@ -822,14 +845,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(s_col + 96, s[3]);
         prepare(s[0], 0);
         prepare(s[1], 1);
-        chunk_max(s[0], s[1], mx);
+        chunk_max(s[0], s[1], mx, 0);
         tmem_ld_wait(s[2]);
         tmem_ld_tie(s[3]);
         prepare(s[2], 2);
         prepare(s[3], 3);
-        chunk_max(s[2], s[3], mx + 4);
+        chunk_max(s[2], s[3], mx + 4, 64);
         const float mx_s = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
-                                 fmaxf(mx[6], mx[7])) * (LOGIT ? 1.f : sl);
+                                 fmaxf(mx[6], mx[7])) * (LOGIT == 0 ? sl : 1.f) +
+                           (LINEAR ? slope2 * (float)(kv0 - qpos) : 0.f);
         // Lazy rescale, decided per row: the reference max moves only when the
         // tile max exceeds it by more than the threshold.  The exponentials
         // start at once with this row's reference; O is rescaled in tensor
@@ -879,8 +903,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // s[c][0..] in order
         const float m_use = (GENERAL && m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t neg2 = f2_pack(-m_use, -m_use);
-        // LOGIT: s already holds scaled logits, so the FMA multiplies by 1
-        const uint64_t mul2 = LOGIT ? f2_pack(1.f, 1.f) : sl2;
+        // INPLACE: s already holds scaled logits, so the FMA multiplies by 1
+        const uint64_t mul2 = INPLACE ? f2_pack(1.f, 1.f) : sl2;
+        // LINEAR: the exponent's addend is slope * (column + kv0 - query) - m
+        const uint64_t am2 = LINEAR ? f2_add(f2_pack(slope2 * (float)(kv0 - qpos), slope2 * (float)(kv0 - qpos)), neg2)
+                                    : neg2;
         uint32_t e4_lo = 0;  // e4m3: the even pair of a word, waiting for the odd one
         // four 32-key quarters; a chunk is 4 / P_CHUNKS consecutive quarters
         constexpr int QPC = 4 / P_CHUNKS;
@@ -888,8 +915,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
+            uint64_t add2 = neg2;
+            if constexpr (LINEAR)
+              add2 = f2_fma(sp2, f2_pack((float)(c * 32 + e), (float)(c * 32 + e + 1)), am2);
             const uint64_t x =
-                f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), mul2, neg2);
+                f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), mul2, add2);
             uint64_t pr;
             if (POLY_EVERY > 0 && ((e >> 1) % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
               pr = exp2_fma_pair(x);

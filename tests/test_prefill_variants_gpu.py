@@ -96,6 +96,18 @@ def test_alibi_per_sequence_and_head(causal):
     assert_matches(inp, causal, alibi_slopes=slopes)
 
 
+@pytest.mark.parametrize("window,d", [((100, 0), 128), ((300, 0), 64), ((0, 0), 128),
+                                      ((-1, 0), 64)])
+def test_alibi_causal_with_left_window(window, d):
+    """Causal ALiBi without softcap (every visible key precedes its query, so
+    the kernel folds the penalty into the row max and the exponent) together
+    with a left window bound, including a window of one key."""
+    lengths = [3, 600, 129, 1000]
+    inp = inputs.make_prefill(lengths, 8, 4, d, True, seed=5450 + d + window[0])
+    slopes = inputs.uniform_slopes((len(lengths), 8), 0.0, 0.3, torch.Generator().manual_seed(5451))
+    assert_matches(inp, True, peaked=window[0] == 0, window=window, alibi_slopes=slopes)
+
+
 @pytest.mark.parametrize("causal,window", [(True, (200, 0)), (False, (64, 300)), (True, (-1, 0))])
 def test_all_variants_together(causal, window):
     lengths = [0, 5, 1200, 129, 640]
