@@ -404,19 +404,22 @@ fa_status fa_prefill_ex(const void* q, const void* k, const void* v, void* o, fl
     return FA_ERR_UNSUPPORTED;
   if (B == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // four kernels per head size: plain causal / full; a band mask alone;
-  // causal ALiBi (no softcap), whose penalty is linear in the key; and a
-  // band with softcap and / or ALiBi, rewriting every score
+  // five kernels per head size: plain causal / full; a band mask alone;
+  // causal ALiBi (no softcap), whose penalty is linear in the key; softcap
+  // without ALiBi, capped inside the exponential loop; and softcap with
+  // ALiBi, or ALiBi under a right bound other than 0, rewriting every score
   const bool gen = var.general();
-  const int logit = (var.softcap > 0.f || var.alibi != nullptr)
-                        ? ((var.alibi != nullptr && var.softcap == 0.f && var.wr == 0) ? 2 : 1)
-                        : 0;
+  const bool cap = var.softcap > 0.f, alibi = var.alibi != nullptr;
+  const int logit = cap ? (alibi ? 1 : 3) : (alibi ? (var.wr == 0 ? 2 : 1) : 0);
   if (d == 64) {
     if (!gen)
       return launch_prefill<64, false>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal, scale, s,
                                        total_tokens, max_seqlen, var);
     if (logit == 1)
       return launch_prefill<64, true, false, 1>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
+                                                scale, s, total_tokens, max_seqlen, var);
+    if (logit == 3)
+      return launch_prefill<64, true, false, 3>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
                                                 scale, s, total_tokens, max_seqlen, var);
     if (logit == 2)
       return launch_prefill<64, true, false, 2>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
@@ -430,6 +433,9 @@ fa_status fa_prefill_ex(const void* q, const void* k, const void* v, void* o, fl
   if (logit == 1)
     return launch_prefill<128, true, false, 1>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
                                                scale, s, total_tokens, max_seqlen, var);
+  if (logit == 3)
+    return launch_prefill<128, true, false, 3>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
+                                              scale, s, total_tokens, max_seqlen, var);
   if (logit == 2)
     return launch_prefill<128, true, false, 2>(q, k, v, o, lse, cu_seqlens, B, Hq, Hkv, causal,
                                                scale, s, total_tokens, max_seqlen, var);

@@ -64,7 +64,10 @@
 // exponent's FMA; 1 rewrites every score in place (softcap, then ALiBi);
 // 2 is ALiBi without softcap under a right bound of 0, where every visible
 // key precedes its query, so the penalty slope * (key - query) is linear in
-// the key's column and joins the row max and the exponent's FMA:
+// the key's column and joins the row max and the exponent's FMA; 3 is
+// softcap without ALiBi: tanh is increasing, so the row max is taken on the
+// raw scores and capped once, and each score is capped inside the
+// exponential loop:
 //   - sliding window (left, right): query i sees keys i-left .. i+right.
 //     Each query tile visits only the K/V tiles that intersect its band
 //     [lo, hi), so a long sequence costs O(L * window), not O(L^2);
@@ -345,6 +348,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   static_assert(GENERAL || LOGIT == 0, "softcap and ALiBi come with the mask-variant kernel");
   constexpr bool INPLACE = LOGIT == 1;  // scores rewritten in place
   constexpr bool LINEAR = LOGIT == 2;   // causal ALiBi folded into max and exponent
+  constexpr bool SOFTCAP = LOGIT == 3;  // softcap applied in the exponential loop
   // one exp2 pair in POLY_EVERY on the FMA pipe, the rest on MUFU (0: all MUFU)
   constexpr int POLY_EVERY = 0;
   extern __shared__ uint8_t smem_raw[];
@@ -851,9 +855,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         prepare(s[2], 2);
         prepare(s[3], 3);
         chunk_max(s[2], s[3], mx + 4, 64);
-        const float mx_s = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
-                                 fmaxf(mx[6], mx[7])) * (LOGIT == 0 ? sl : 1.f) +
-                           (LINEAR ? slope2 * (float)(kv0 - qpos) : 0.f);
+        float mx_s = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
+                           fmaxf(mx[6], mx[7]));
+        if constexpr (LOGIT == 0) mx_s *= sl;
+        if constexpr (LINEAR) mx_s += slope2 * (float)(kv0 - qpos);
+        if constexpr (SOFTCAP)
+          mx_s = mx_s == -INFINITY ? -INFINITY : softcap_log2(mx_s, p.cap_in, p.cap_out);
         // Lazy rescale, decided per row: the reference max moves only when the
         // tile max exceeds it by more than the threshold.  The exponentials
         // start at once with this row's reference; O is rescaled in tensor
@@ -905,6 +912,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t neg2 = f2_pack(-m_use, -m_use);
         // INPLACE: s already holds scaled logits, so the FMA multiplies by 1
         const uint64_t mul2 = INPLACE ? f2_pack(1.f, 1.f) : sl2;
+        const uint64_t cap2 = f2_pack(p.cap_out, p.cap_out);  // SOFTCAP
         // LINEAR: the exponent's addend is slope * (column + kv0 - query) - m
         const uint64_t am2 = LINEAR ? f2_add(f2_pack(slope2 * (float)(kv0 - qpos), slope2 * (float)(kv0 - qpos)), neg2)
                                     : neg2;
@@ -915,11 +923,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            uint64_t add2 = neg2;
-            if constexpr (LINEAR)
-              add2 = f2_fma(sp2, f2_pack((float)(c * 32 + e), (float)(c * 32 + e + 1)), am2);
-            const uint64_t x =
-                f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), mul2, add2);
+            uint64_t x;
+            if constexpr (SOFTCAP) {
+              // cap * tanh, in log2 units, minus m; a masked score stays -inf
+              const float s0 = __uint_as_float(s[c][e]), s1 = __uint_as_float(s[c][e + 1]);
+              const uint64_t th = f2_fma(f2_pack(rcp_approx(1.f + ex2(s0 * p.cap_in)),
+                                                 rcp_approx(1.f + ex2(s1 * p.cap_in))),
+                                         f2_pack(-2.f, -2.f), f2_pack(1.f, 1.f));
+              float x0, x1;
+              f2_unpack(f2_fma(th, cap2, neg2), x0, x1);
+              x = f2_pack(s0 == -INFINITY ? -INFINITY : x0, s1 == -INFINITY ? -INFINITY : x1);
+            } else {
+              uint64_t add2 = neg2;
+              if constexpr (LINEAR)
+                add2 = f2_fma(sp2, f2_pack((float)(c * 32 + e), (float)(c * 32 + e + 1)), am2);
+              x = f2_fma(f2_pack(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), mul2, add2);
+            }
             uint64_t pr;
             if (POLY_EVERY > 0 && ((e >> 1) % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
               pr = exp2_fma_pair(x);

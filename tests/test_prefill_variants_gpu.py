@@ -81,6 +81,16 @@ def test_softcap(softcap, scale, causal):
     assert_matches(inp, causal, peaked=scale == 1.0 and softcap > 8, softcap=softcap)
 
 
+@pytest.mark.parametrize("causal,window,d", [(True, (150, 0), 128), (False, (40, 260), 64),
+                                             (True, (-1, 0), 64), (False, (0, 0), 128)])
+def test_softcap_with_window(causal, window, d):
+    """Softcap without ALiBi (the kernel caps each score inside its
+    exponential loop and the row max once) under band masks, so masked
+    scores must stay at zero weight."""
+    inp = inputs.make_prefill([2, 300, 129, 900], 8, 2, d, causal, seed=5350 + d + window[0])
+    assert_matches(inp, causal, peaked=window == (0, 0), window=window, softcap=5.0)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_alibi_per_head(causal, d):
