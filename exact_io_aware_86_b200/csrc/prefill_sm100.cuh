@@ -79,7 +79,7 @@
 // starts inside the tile), so its running max may start at -inf; the exp
 // argument and the rescale factor are guarded for that.
 //
-// FP8 (a third instantiation, FP8 = true; causal or full mask): Q, K and V
+// FP8 (an instantiation of its own, FP8 = true; causal or full mask): Q, K, V
 // are e4m3 bytes with per-tensor descale factors.  Both products run as
 // tcgen05 kind::f8f6f4 MMAs (K steps of 32 elements = 32 bytes, so a d=128
 // row is one 128-byte swizzle panel and a tile is 16 KB).  P is rounded to
