@@ -107,6 +107,29 @@ def test_fp8_workload_every_pair():
     check_rows(inp, o, lse, loose=True)
 
 
+def _random_case(i):
+    """Configuration i of a seeded random sweep (a pure function of i): 1-4
+    packed sequences of 1-400 tokens, GQA groups 1-8, causal or full, and
+    per-tensor spreads that the descales bring back to unit scale."""
+    rng = np.random.default_rng(7400 + i)
+    lengths = [int(rng.integers(1, 400)) for _ in range(int(rng.integers(1, 5)))]
+    Hkv = int(rng.choice([1, 2, 4]))
+    group = int(rng.choice([1, 2, 4, 8]))
+    causal = bool(rng.random() < 0.6)
+    spread = tuple(float(x) for x in rng.choice([0.5, 1.0, 4.0, 16.0], size=3))
+    return lengths, Hkv * group, Hkv, causal, spread
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_random_configuration(i):
+    lengths, Hq, Hkv, causal, spread = _random_case(i)
+    inp = inputs.make_prefill_fp8(lengths, Hq, Hkv, 128, causal, seed=7500 + i, spread=spread)
+    o, lse = run(inp)
+    # the exact form of the bound holds an L x L x d array per pair: the
+    # triangle-inequality form above 256 tokens
+    check_rows(inp, o, lse, loose=max(lengths) > 256)
+
+
 def test_rejects_bad_descale_and_head_dim():
     inp = inputs.make_prefill_fp8([16], 2, 2, 128, True, seed=7300)
     q, k, v, cu = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.cu_seqlens))
