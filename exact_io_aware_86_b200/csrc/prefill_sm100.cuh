@@ -782,8 +782,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           need_mask = kv0 + BN > len || (p.causal && kv0 + BN - 1 > rs);
           lim_hi = min(len, p.causal ? qpos + 1 : len) - kv0;
         }
-        // softcap or ALiBi: logits in log2 units (optional cap, then the
-        // ALiBi penalty); then the mask (band, sequence end, causal)
+        // INPLACE (softcap with ALiBi, or ALiBi under a right bound other
+        // than 0): logits in log2 units (optional cap, then the ALiBi
+        // penalty); then, in every kernel, the mask (band, sequence end,
+        // causal)
         auto prepare = [&](uint32_t (&x)[32], int c) {
           if constexpr (INPLACE) {
             if (p.cap_out > 0.f) {
